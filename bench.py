@@ -1,0 +1,430 @@
+"""Benchmark of the HGA routed-attention hot path on B200.
+
+One step = one pass of the whole path over the query segment of the
+Qwen3-30B-A3B-shaped 64K workload (32 query heads, 4 KV heads, d=128, bf16,
+last 2048 of 65536 tokens as 32 query blocks, sink 64, local 512, top-32
+chunks then top-64 groups): summaries of the segment's chunks/groups, chunk
+routing, group routing and gathered exact-token attention.  The 64K history
+(K/V and its summaries) is committed once before timing, like a KV cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hga|reference]
+
+Prints one JSON line (rank 0).  N > 1 runs independent replicas, one per GPU
+(the path has no exchange step), timed as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import hga_inputs as gi  # noqa: E402
+
+METRIC = "routed-attn query tokens/s @64K ctx; % of HBM/tensor roofline"
+UNIT = "query tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- dist
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(
+            "nccl" if torch.cuda.is_available() else "gloo",
+            timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"hga_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- workload
+
+def algorithmic_counts(w: gi.Workload, group_cnt: np.ndarray):
+    """Exact algorithmic work of one pass from the routed counts.
+    attention flops: 4*d per (query row, attended token), causal-exact;
+    routing flops: 2*d per (query row, candidate summary);
+    attention bytes: Q + O once, plus the routed K/V working set per
+    (block, KV head), plus summaries read."""
+    d, G, B, g, C = w.head_dim, w.G, w.qblock, w.group, w.chunk
+    nb = -(-w.Tq // B)
+    att_pairs = 0
+    ws_tokens = 0
+    route_chunk_pairs = 0
+    route_group_pairs = 0
+    for b in range(nb):
+        b0 = w.q0 + b * B
+        b1 = min(b0 + B, w.T)
+        sink = min(w.sink, b0)
+        loc = b0 - max(sink, b0 - w.local)
+        hi = (b0 - w.local) // C if b0 - w.local > 0 else 0
+        n_cand = max(0, hi - w.sink // C)
+        kc = n_cand if w.top_chunks <= 0 else min(w.top_chunks, n_cand)
+        for h in range(w.n_kv_heads):
+            routed = int(group_cnt[h, b]) * g
+            hist = sink + routed + loc
+            for pos in range(b0, b1):
+                att_pairs += G * (hist + pos - b0 + 1)
+            ws_tokens += hist + (b1 - b0)
+            route_chunk_pairs += (b1 - b0) * G * n_cand
+            route_group_pairs += (b1 - b0) * G * kc * (C // g)
+    esz = 2 if w.dtype == "bf16" else 4
+    att_flops = 4 * d * att_pairs
+    att_bytes = (2 * w.Tq * w.n_q_heads * d + ws_tokens * 2 * d) * esz
+    return {"attn_flops": att_flops, "attn_bytes": att_bytes,
+            "route_chunk_flops": 2 * d * route_chunk_pairs,
+            "route_group_flops": 2 * d * route_group_pairs,
+            "density": att_pairs / (G * w.n_kv_heads * sum(
+                p + 1 for p in range(w.q0, w.T)))}
+
+
+def dense_sdpa_time(w, q, k, v, steps=5):
+    """Same-shape dense causal attention (torch SDPA, bf16, bottom-right
+    causal alignment for a query segment at the end of the context)."""
+    from torch.nn.attention.bias import causal_lower_right
+    qt = q.permute(1, 0, 2).unsqueeze(0)
+    kt = k[:, :w.T].unsqueeze(0)
+    vt = v[:, :w.T].unsqueeze(0)
+    mask = causal_lower_right(w.Tq, w.T)
+    f = lambda: torch.nn.functional.scaled_dot_product_attention(
+        qt, kt, vt, attn_mask=mask, enable_gqa=True)
+    try:
+        f()
+    except RuntimeError:
+        rep = w.G
+        kt = kt.repeat_interleave(rep, dim=1)
+        vt = vt.repeat_interleave(rep, dim=1)
+        f = lambda: torch.nn.functional.scaled_dot_product_attention(
+            qt, kt, vt, attn_mask=mask)
+        f()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        f()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def cpu_baseline(w: gi.Workload, inp: gi.Inputs, budget_s: float = 15.0):
+    """The oracle as it stands, on this host's cores, over a bounded sample of
+    the workload's (block, KV head) units (plus the summaries it needs)."""
+    from oracle import hga_oracle as ho
+    p = ho.Params(w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.group,
+                  w.qblock, w.sink, w.local, w.top_chunks, w.top_groups, w.dtype)
+    cores = len(os.sched_getaffinity(0))
+    t0 = time.perf_counter()
+    q = gi.to_f64(inp.q)
+    k = gi.to_f64(inp.k)
+    v = gi.to_f64(inp.v)
+    csum, gsum = ho.build_summaries(k, p, 0, w.T)
+    t_setup = time.perf_counter() - t0
+    nb = -(-w.Tq // w.qblock)
+    units = [(b, h) for b in range(nb) for h in range(w.n_kv_heads)]
+    done = 0
+    t1 = time.perf_counter()
+    for (b, h) in units:
+        ho.hga_forward(q, k, v, w.q0, p, units=[(b, h)], csum=csum, gsum=gsum)
+        done += 1
+        if time.perf_counter() - t1 > budget_s:
+            break
+    dt = time.perf_counter() - t1
+    q_tokens = done * w.qblock / w.n_kv_heads     # one unit = 64 positions x 1/Hkv of the heads
+    return {"value": q_tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {len(units)} (block, KV head) units of {w.name} "
+                      f"(routing + attention, float64 NumPy); history summaries "
+                      f"({t_setup:.1f} s) excluded as commit cost"}
+
+
+# ---------------------------------------------------------------- main arm
+
+def run_hga(args, world, rank, local):
+    from long_context_hga_b200 import hga
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = gi.WORKLOADS[args.workload]
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    q = inp.q.to(dev)
+    k = inp.k.to(dev)
+    v = inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    stream = torch.cuda.current_stream()
+    # commit the history once (setup, not timed)
+    hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)
+        hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt)
+        hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt,
+                         bufs.group_idx, bufs.group_cnt)
+        hga.attend(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert hga.check() == 0
+    counts = algorithmic_counts(w, bufs.group_cnt.cpu().numpy())
+
+    n_kern = 4
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_kern + 1)]
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = hga.launch_count()
+    t_wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.zero_()                      # cold L2, outside the events
+        e = ev[i]
+        e[0].record(stream)
+        hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)
+        e[1].record(stream)
+        hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt)
+        e[2].record(stream)
+        hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt,
+                         bufs.group_idx, bufs.group_cnt)
+        e[3].record(stream)
+        hga.attend(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
+        e[4].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    t_wall = time.perf_counter() - t_wall0
+    launches = hga.launch_count() - launches0
+    clk = clocks.stop()
+    per_kernel = np.array([[ev[i][j].elapsed_time(ev[i][j + 1]) for j in range(n_kern)]
+                           for i in range(args.steps)])          # ms
+    step_ms = per_kernel.sum(axis=1)
+    ms_local = float(step_ms.mean())
+    ms = max_over_ranks(ms_local, world, dev)
+    assert hga.check() == 0
+
+    # end-to-end through the public API with host buffers: pinned host Q and
+    # the segment's K/V in, O out, copies inside the timed region
+    q_h = inp.q.pin_memory()
+    kseg_h = inp.k[:, w.q0:].contiguous().pin_memory()
+    vseg_h = inp.v[:, w.q0:].contiguous().pin_memory()
+    o_h = torch.empty(bufs.o.shape, dtype=bufs.o.dtype).pin_memory()
+    q_d = torch.empty_like(q)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        k[:, w.q0:].copy_(kseg_h, non_blocking=True)
+        v[:, w.q0:].copy_(vseg_h, non_blocking=True)
+        hga.forward(p, q_d, w.q0, k, v, bufs)
+        o_h.copy_(bufs.o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, args.steps)
+    es.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ee.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(es.elapsed_time(ee) / e2e_steps, world, dev)
+    h2d = q_h.numel() * q_h.element_size() + 2 * kseg_h.numel() * kseg_h.element_size()
+    d2h = o_h.numel() * o_h.element_size()
+
+    dense_ms = None
+    if not args.no_dense:
+        try:
+            dense_ms = dense_sdpa_time(w, q, k, v)
+        except Exception as exc:  # comparator only
+            print(f"dense comparator failed: {exc}", file=sys.stderr)
+
+    peaks, peak_kind = load_peaks()
+    att_ms = float(per_kernel[:, 3].mean())
+    att_tflops = counts["attn_flops"] / (att_ms * 1e-3) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    out = None
+    if rank == 0:
+        n_tok = w.Tq * world
+        value = n_tok / (ms * 1e-3)
+        kernels = {name: round(float(per_kernel[:, j].mean()) * 1e3, 2) for j, name in
+                   enumerate(["build_summaries", "route_chunks", "route_groups", "attend"])}
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded N(0,1) Q/K/V, RoPE, planted needles)",
+            "config": {"workload": w.name, "T": w.T, "q0": w.q0, "query_tokens": w.Tq,
+                       "heads": f"{w.n_q_heads}q/{w.n_kv_heads}kv", "head_dim": w.head_dim,
+                       "routing": f"chunk {w.chunk}, group {w.group}, sink {w.sink}, "
+                                  f"local {w.local}, top {w.top_chunks} chunks / "
+                                  f"{w.top_groups} groups",
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed (256 MiB write) before every step, outside the events"},
+            "kernel_us": kernels,
+            "attn_tflops": att_tflops,
+            "route_tflops": (counts["route_chunk_flops"] + counts["route_group_flops"]) /
+                            (float(per_kernel[:, 1:3].sum(axis=1).mean()) * 1e-3) / 1e12,
+            "density": counts["density"],
+            "roofline": {"bound": "tensor", "kernel": "hga_attend",
+                         "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": att_tflops / peak_tf, "traffic": None,
+                         "peak_source": f"{peak_kind} bf16 burst",
+                         "algorithmic_flops": counts["attn_flops"],
+                         "algorithmic_bytes": counts["attn_bytes"],
+                         "hbm_frac": counts["attn_bytes"] / (att_ms * 1e-3) / 1e9 /
+                                     peaks["hbm_gbs"]},
+            "e2e": {"value": n_tok / (e2e_ms * 1e-3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "dense_sdpa": None if dense_ms is None else {
+                "value": w.Tq / (dense_ms * 1e-3), "unit": UNIT, "ms": dense_ms},
+            "wall_s_timed_region": t_wall,
+        }
+    return out, w, inp
+
+
+def run_reference(args, world, rank):
+    """The oracle as the reference arm: CPU, host cores, bounded sample."""
+    if rank != 0:
+        return None
+    w = gi.WORKLOADS[args.workload]
+    inp = gi.make_inputs(w)
+    vals = []
+    info = None
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        info = cpu_baseline(w, inp, budget_s=per_step)
+        if i >= args.warmup:
+            vals.append(info["value"])
+    v = float(np.mean(vals))
+    return {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": w.Tq / v * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) Q/K/V, RoPE, planted needles)",
+            "config": {"workload": w.name}, "impl": "reference",
+            "cpu_baseline": dict(info, value=v),
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
+    ap.add_argument("--workload", default=gi.QWEN3_30B_64K.name, choices=sorted(gi.WORKLOADS))
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "hga":
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        out = run_reference(args, world, rank)
+    else:
+        out, w, inp = run_hga(args, world, rank, local)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_seconds)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

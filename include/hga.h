@@ -1,0 +1,181 @@
+/*
+ * hga.h - C ABI of the HGA routed-attention library (libhga.so, sm_100a).
+ *
+ * Hierarchical Global Attention (HGA), exact-token two-level routed causal
+ * attention for one layer's projected, RoPE-applied Q/K/V, as described on the
+ * page "Long-Context Fine-Tuning with Limited VRAM", section 2.1 ("Exact-token
+ * hierarchical routing"):
+ *   1. a summary for every closed 64-token chunk and every 8-token group of
+ *      the keys                                      -> hga_build_summaries
+ *   2. each 64-query block scores the chunk summaries and keeps the best
+ *      chunks, besides fixed sink and local windows  -> hga_route_chunks
+ *   3. the kept chunks are opened and the best 8-token groups inside them are
+ *      kept                                          -> hga_route_groups
+ *   4. softmax attention over the exact token K/V of the kept groups, the
+ *      sink, the local window and the causal diagonal -> hga_attend
+ * Section 6.1 of the same page notes that one routing decision serves every
+ * query of a block: routing is per (query block, KV head).
+ *
+ * Readings this library fixes where the pages are silent:
+ *   - summary = mean of the post-RoPE keys, accumulated exactly (float64) and
+ *     rounded once, to nearest even, to the storage dtype;
+ *   - block score of a summary s = max over the block's queries and the query
+ *     heads sharing the KV head of q.s/sqrt(d) (ranking uses q.s);
+ *   - candidate chunks of the block at b0: sink/chunk <= c < (b0-local)/chunk;
+ *   - local window = tokens [b0-local, b0) plus the block's causal diagonal;
+ *     sink = tokens [0, sink);
+ *   - top-k keeps the first min(k, n) candidates by (score desc, index asc);
+ *     k <= 0 keeps all; the group budget is global over the kept chunks.
+ *
+ * Layouts (all row-major, element type = params.dtype):
+ *   q, o        [n_q][n_q_heads][head_dim]          query i is position q_start+i
+ *   k, v        [n_kv_heads][t_cap][head_dim]       token t of head h at (h*t_cap+t)*d
+ *   chunk_sum   [n_kv_heads][t_cap/chunk][head_dim]
+ *   group_sum   [n_kv_heads][t_cap/group][head_dim]
+ *   chunk_idx   [n_kv_heads][n_blocks][cap_c]  int32, cap_c = hga_index_capacity(p,t_cap,0)
+ *   chunk_cnt   [n_kv_heads][n_blocks]         int32
+ *   group_idx   [n_kv_heads][n_blocks][cap_g]  int32, cap_g = hga_index_capacity(p,t_cap,1)
+ *   group_cnt   [n_kv_heads][n_blocks]         int32
+ *   lse         [n_q][n_q_heads] float32 (natural log), optional
+ * with n_blocks = ceil(n_q / qblock).  The context of a call is T = q_start + n_q
+ * tokens; queries attend only to tokens < T (causal).
+ *
+ * Ownership: the caller owns every buffer (device memory unless stated); the
+ * library never allocates or frees and keeps no per-call state.  Inputs are
+ * read-only.  Index outputs are fully overwritten: unused slots become -1 and
+ * lists are in ascending order.  Summary outputs are written only for the
+ * chunks/groups the call covers.
+ *
+ * Errors: every call is asynchronous on `stream`.  Argument errors are
+ * detected on the host and returned before anything is launched.  Launch
+ * failures return HGA_ERR_CUDA.  Errors found by a kernel (an index list entry
+ * outside the legal range, for example) are recorded in a device status word
+ * and returned by hga_check(); kernels never trap.
+ *
+ * Supported: dtype bf16 (tensor-core path) or fp32 (exact FFMA path);
+ * head_dim 64 or 128; chunk 64, group 8, qblock 64; sink and local multiples
+ * of chunk; n_q_heads a multiple of n_kv_heads.
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hga_stream_t;   /* same object as cudaStream_t */
+
+typedef enum {
+  HGA_OK = 0,
+  HGA_ERR_INVALID_ARG = 1,   /* bad pointer, size, alignment or parameter      */
+  HGA_ERR_UNSUPPORTED = 2,   /* legal but not built: dtype, head_dim, sizes     */
+  HGA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed            */
+  HGA_ERR_DEVICE_CHECK = 4,  /* a kernel found an out-of-range index (hga_check)*/
+  HGA_ERR_TIMEOUT = 5        /* a bounded device wait gave up (hga_check)       */
+} hga_status;
+
+typedef enum { HGA_BF16 = 0, HGA_FP32 = 1 } hga_dtype;
+
+typedef struct hga_params {
+  int32_t n_q_heads;    /* query heads; a multiple of n_kv_heads              */
+  int32_t n_kv_heads;   /* key/value heads (GQA)                              */
+  int32_t head_dim;     /* 64 or 128                                          */
+  int32_t chunk;        /* chunk size in tokens (64)                          */
+  int32_t group;        /* group size in tokens (8)                           */
+  int32_t qblock;       /* query block size (64)                              */
+  int32_t sink;         /* sink window, tokens [0, sink); multiple of chunk   */
+  int32_t local;        /* local window before each block; multiple of chunk  */
+  int32_t top_chunks;   /* chunk budget per (block, KV head); <= 0 = all       */
+  int32_t top_groups;   /* group budget per (block, KV head); <= 0 = all       */
+  int32_t dtype;        /* hga_dtype of q, k, v, o and the summaries          */
+} hga_params;
+
+/* Step 1 (section 2.1, "HGA builds two levels of key summaries from the
+ * model's existing projected keys").  For every KV head h writes
+ *   chunk_sum[h][c] = mean(k[h][c*chunk .. c*chunk+chunk-1])
+ * for each chunk c with t_begin <= c*chunk and (c+1)*chunk <= t_end, and
+ *   group_sum[h][j] = mean(k[h][j*group .. j*group+group-1])
+ * for each group j with t_begin <= j*group and (j+1)*group <= t_end.
+ * The mean is exact before a single round-to-nearest-even to the dtype.
+ * Requires t_begin % chunk == 0 and 0 <= t_begin <= t_end <= t_cap. */
+hga_status hga_build_summaries(const hga_params* p, const void* k,
+                               int64_t t_cap, int64_t t_begin, int64_t t_end,
+                               void* chunk_sum, void* group_sum,
+                               hga_stream_t stream);
+
+/* Step 2 (section 2.1, "Chunk selection").  For each query block b (queries
+ * q_start + b*qblock ...) and KV head h: scores every candidate chunk
+ * (sink/chunk <= c < (b0-local)/chunk) by the max over the block's rows of
+ * q.chunk_sum[h][c], keeps min(top_chunks, n) by (score desc, index asc) and
+ * writes them ascending to chunk_idx[h][b][:], the count to chunk_cnt[h][b].
+ * chunk_sum must hold every candidate (built with t_end >= q_start).
+ * Requires q_start % qblock == 0 and q_start + n_q <= t_cap. */
+hga_status hga_route_chunks(const hga_params* p, const void* q,
+                            int64_t q_start, int64_t n_q,
+                            const void* chunk_sum, int64_t t_cap,
+                            int32_t* chunk_idx, int32_t* chunk_cnt,
+                            hga_stream_t stream);
+
+/* Step 3 (section 2.1, "Group selection").  Candidates of (b, h) are the
+ * chunk/group groups of every chunk in chunk_idx[h][b][0 .. chunk_cnt-1];
+ * scored as in step 2 against group_sum; keeps min(top_groups, n) and writes
+ * them ascending to group_idx[h][b][:], the count to group_cnt[h][b].
+ * chunk_idx/chunk_cnt are the outputs of hga_route_chunks for the same
+ * q_start/n_q/t_cap.  An out-of-range chunk index sets HGA_ERR_DEVICE_CHECK
+ * (read by hga_check) and is skipped. */
+hga_status hga_route_groups(const hga_params* p, const void* q,
+                            int64_t q_start, int64_t n_q,
+                            const void* group_sum, int64_t t_cap,
+                            const int32_t* chunk_idx, const int32_t* chunk_cnt,
+                            int32_t* group_idx, int32_t* group_cnt,
+                            hga_stream_t stream);
+
+/* Step 4 (section 2.1, "Exact-token attention": only exact token K/V, never
+ * summaries).  Query at position pos (block start b0, query head hq, KV head
+ * h = hq / (n_q_heads/n_kv_heads)) attends the set
+ *   [0, min(sink, pos+1))  U  tokens of group_idx[h][b][0..group_cnt-1]
+ *   U  [max(0, b0-local), b0)  U  [b0, pos]
+ * with softmax(q.k/sqrt(d)) and writes o (dtype) and, when lse != NULL, the
+ * natural-log sum of exponentials of the scaled scores.  Group indices outside
+ * the legal range set HGA_ERR_DEVICE_CHECK and are skipped. */
+hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start,
+                      int64_t n_q, const void* k, const void* v, int64_t t_cap,
+                      const int32_t* group_idx, const int32_t* group_cnt,
+                      void* o, float* lse, hga_stream_t stream);
+
+/* Steps 1-4 in one call for a query segment whose own K/V already sit in
+ * k/v at [q_start, q_start+n_q): builds the summaries of the segment's
+ * closed chunks/groups, then routes and attends.  Index buffers as above. */
+hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start,
+                       int64_t n_q, const void* k, const void* v,
+                       int64_t t_cap, void* chunk_sum, void* group_sum,
+                       int32_t* chunk_idx, int32_t* chunk_cnt,
+                       int32_t* group_idx, int32_t* group_cnt, void* o,
+                       float* lse, hga_stream_t stream);
+
+/* Slots per (KV head, block) of chunk_idx (which = 0) or group_idx
+ * (which = 1) for a context capacity t_cap; -1 on invalid parameters. */
+int64_t hga_index_capacity(const hga_params* p, int64_t t_cap, int32_t which);
+
+/* Validates a parameter block without launching anything. */
+hga_status hga_validate_params(const hga_params* p);
+
+/* Synchronises `stream`, then returns and clears the device status word
+ * (HGA_OK, HGA_ERR_DEVICE_CHECK or HGA_ERR_TIMEOUT), or HGA_ERR_CUDA when the
+ * synchronisation itself fails. */
+hga_status hga_check(hga_stream_t stream);
+
+/* Static string naming a status code. */
+const char* hga_status_string(hga_status s);
+
+/* Number of kernel launches issued by this library since load (for
+ * accounting in benchmarks); never reset. */
+int64_t hga_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HGA_H */

@@ -1,0 +1,305 @@
+// libhga: C ABI entry points (declared in include/hga.h).  Host-side argument
+// checks, launch sizing and the device status word; the kernels live in the
+// included .cuh files.  One translation unit so that the status word is a
+// single device symbol without relocatable device code.
+#include <atomic>
+#include <cstdio>
+
+#include "hga.h"
+#include "common.cuh"
+#include "summaries.cuh"
+#include "route.cuh"
+#include "attend.cuh"
+
+namespace {
+
+std::atomic<int64_t> g_launches{0};
+
+inline hga_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
+
+inline hga_status after_launch() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cuda_ok(cudaGetLastError());
+}
+
+// Opt every kernel into the full 227 KB of dynamic shared memory once per
+// device (the attribute is per device context).
+template <auto kernel>
+hga_status allow_smem(size_t bytes) {
+  static std::atomic<uint64_t> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HGA_ERR_CUDA;
+  if (bytes > 227 * 1024) return HGA_ERR_UNSUPPORTED;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return HGA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+      cudaSuccess)
+    return HGA_ERR_CUDA;
+  done.fetch_or(bit, std::memory_order_acq_rel);
+  return HGA_OK;
+}
+
+hga_status check_params(const hga_params* p) {
+  if (!p) return HGA_ERR_INVALID_ARG;
+  if (p->n_q_heads <= 0 || p->n_kv_heads <= 0 || p->n_q_heads % p->n_kv_heads) return HGA_ERR_INVALID_ARG;
+  if (p->head_dim <= 0 || p->chunk <= 0 || p->group <= 0 || p->qblock <= 0) return HGA_ERR_INVALID_ARG;
+  if (p->chunk % p->group) return HGA_ERR_INVALID_ARG;
+  if (p->sink < 0 || p->local < 0 || p->sink % p->chunk || p->local % p->chunk) return HGA_ERR_INVALID_ARG;
+  if (p->dtype != HGA_BF16 && p->dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return HGA_ERR_UNSUPPORTED;
+  if (p->chunk != 64 || p->group != 8 || p->qblock != 64) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+inline int64_t cap_chunks(const hga_params* p, int64_t t_cap) {
+  const int64_t n = t_cap / p->chunk;
+  return p->top_chunks > 0 ? std::min<int64_t>(p->top_chunks, n) : n;
+}
+inline int64_t cap_groups(const hga_params* p, int64_t t_cap) {
+  const int64_t n = cap_chunks(p, t_cap) * (p->chunk / p->group);
+  return p->top_groups > 0 ? std::min<int64_t>(p->top_groups, n) : n;
+}
+
+hga_status check_segment(const hga_params* p, int64_t q_start, int64_t n_q, int64_t t_cap) {
+  if (q_start < 0 || n_q < 0 || t_cap <= 0) return HGA_ERR_INVALID_ARG;
+  if (q_start % p->qblock) return HGA_ERR_INVALID_ARG;
+  if (q_start + n_q > t_cap) return HGA_ERR_INVALID_ARG;
+  if ((n_q + p->qblock - 1) / p->qblock > 65535) return HGA_ERR_UNSUPPORTED;
+  return HGA_OK;
+}
+
+constexpr int kMaxRouteCands = 16384;
+constexpr int kMaxKeptChunks = 2048;
+
+template <typename T, int D>
+hga_status launch_route(hga::RouteArgs& a, cudaStream_t st) {
+  const size_t smem = hga::route_smem_bytes<T, D>(a.max_cands);
+  hga_status s = allow_smem<hga::route_kernel<T, D>>(smem);
+  if (s != HGA_OK) return s;
+  dim3 grid(a.n_blocks, a.Hkv);
+  hga::route_kernel<T, D><<<grid, hga::kRouteThreads, smem, st>>>(a);
+  return after_launch();
+}
+
+hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                        const void* summ, int64_t t_cap, const int32_t* in_idx,
+                        const int32_t* in_cnt, int32_t* out_idx, int32_t* out_cnt, int group_mode,
+                        cudaStream_t st) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!q || !summ || !out_idx || !out_cnt || (group_mode && (!in_idx || !in_cnt)))
+    return HGA_ERR_INVALID_ARG;
+  hga::RouteArgs a{};
+  a.q = q;
+  a.q_start = q_start;
+  a.n_q = n_q;
+  a.summ = summ;
+  a.n_blocks = (int)((n_q + p->qblock - 1) / p->qblock);
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.G = p->n_q_heads / p->n_kv_heads;
+  a.chunk = p->chunk;
+  a.group = p->group;
+  a.qblock = p->qblock;
+  a.sink = p->sink;
+  a.local = p->local;
+  a.group_mode = group_mode;
+  a.in_idx = in_idx;
+  a.in_cnt = in_cnt;
+  a.out_idx = out_idx;
+  a.out_cnt = out_cnt;
+  const int per = p->chunk / p->group;
+  if (!group_mode) {
+    a.n_summ_cap = t_cap / p->chunk;
+    a.in_cap = 0;
+    a.out_cap = cap_chunks(p, t_cap);
+    a.top_k = p->top_chunks;
+    const int64_t last_b0 = q_start + (int64_t)(a.n_blocks - 1) * p->qblock;
+    const int64_t hi = last_b0 - p->local > 0 ? (last_b0 - p->local) / p->chunk : 0;
+    const int64_t n = std::max<int64_t>(0, hi - p->sink / p->chunk);
+    if (n > kMaxRouteCands) return HGA_ERR_UNSUPPORTED;
+    a.max_cands = (int)std::max<int64_t>(n, 1);
+  } else {
+    a.n_summ_cap = t_cap / p->group;
+    a.in_cap = cap_chunks(p, t_cap);
+    a.out_cap = cap_groups(p, t_cap);
+    a.top_k = p->top_groups;
+    if (a.in_cap > kMaxKeptChunks || a.in_cap * per > kMaxRouteCands) return HGA_ERR_UNSUPPORTED;
+    a.max_cands = (int)std::max<int64_t>(a.in_cap * per, 1);
+  }
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? launch_route<__nv_bfloat16, 128>(a, st)
+                              : launch_route<__nv_bfloat16, 64>(a, st);
+  return p->head_dim == 128 ? launch_route<float, 128>(a, st) : launch_route<float, 64>(a, st);
+}
+
+template <typename T, int D>
+hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_begin, int64_t t_end,
+                            int chunk, int group, void* cs, void* gs, cudaStream_t st) {
+  const int64_t c_first = t_begin / chunk;
+  const int64_t c_last = (t_end + chunk - 1) / chunk;   // partial chunk: its closed groups
+  const int64_t n_chunks = c_last - c_first;
+  if (n_chunks <= 0) return HGA_OK;
+  const int64_t warps = (int64_t)Hkv * n_chunks;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffff) return HGA_ERR_UNSUPPORTED;
+  hga::summaries_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
+      reinterpret_cast<const T*>(k), t_cap, Hkv, c_first, n_chunks, t_end, chunk, group,
+      reinterpret_cast<T*>(cs), reinterpret_cast<T*>(gs));
+  return after_launch();
+}
+
+template <int D>
+hga_status launch_attend_bf16(hga::AttendArgs& a, cudaStream_t st) {
+  const size_t smem = hga::attend_mma_smem_bytes<D>(a.max_list);
+  hga_status s = allow_smem<hga::attend_mma_kernel<D>>(smem);
+  if (s != HGA_OK) return s;
+  dim3 grid((a.qblock * a.G + hga::kAttRows - 1) / hga::kAttRows, a.n_blocks, a.Hkv);
+  hga::attend_mma_kernel<D><<<grid, 128, smem, st>>>(a);
+  return after_launch();
+}
+
+template <int D>
+hga_status launch_attend_f32(hga::AttendArgs& a, cudaStream_t st) {
+  const size_t smem = (size_t)a.max_list * 4;
+  hga_status s = allow_smem<hga::attend_f32_kernel<D>>(smem);
+  if (s != HGA_OK) return s;
+  dim3 grid((a.qblock * a.G + hga::kAttF32Rows - 1) / hga::kAttF32Rows, a.n_blocks, a.Hkv);
+  hga::attend_f32_kernel<D><<<grid, 256, smem, st>>>(a);
+  return after_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+hga_status hga_validate_params(const hga_params* p) { return check_params(p); }
+
+int64_t hga_index_capacity(const hga_params* p, int64_t t_cap, int32_t which) {
+  if (check_params(p) != HGA_OK || t_cap < 0) return -1;
+  if (which == 0) return cap_chunks(p, t_cap);
+  if (which == 1) return cap_groups(p, t_cap);
+  return -1;
+}
+
+hga_status hga_build_summaries(const hga_params* p, const void* k, int64_t t_cap,
+                               int64_t t_begin, int64_t t_end, void* chunk_sum,
+                               void* group_sum, hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if (t_cap <= 0 || t_begin < 0 || t_begin > t_end || t_end > t_cap) return HGA_ERR_INVALID_ARG;
+  if (t_begin % p->chunk) return HGA_ERR_INVALID_ARG;
+  if (t_begin == t_end) return HGA_OK;
+  if (!k || !chunk_sum || !group_sum) return HGA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int Hkv = p->n_kv_heads;
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128
+               ? launch_summaries<__nv_bfloat16, 128>(k, t_cap, Hkv, t_begin, t_end, p->chunk,
+                                                      p->group, chunk_sum, group_sum, st)
+               : launch_summaries<__nv_bfloat16, 64>(k, t_cap, Hkv, t_begin, t_end, p->chunk,
+                                                     p->group, chunk_sum, group_sum, st);
+  return p->head_dim == 128
+             ? launch_summaries<float, 128>(k, t_cap, Hkv, t_begin, t_end, p->chunk, p->group,
+                                            chunk_sum, group_sum, st)
+             : launch_summaries<float, 64>(k, t_cap, Hkv, t_begin, t_end, p->chunk, p->group,
+                                           chunk_sum, group_sum, st);
+}
+
+hga_status hga_route_chunks(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                            const void* chunk_sum, int64_t t_cap, int32_t* chunk_idx,
+                            int32_t* chunk_cnt, hga_stream_t stream) {
+  return route_common(p, q, q_start, n_q, chunk_sum, t_cap, nullptr, nullptr, chunk_idx,
+                      chunk_cnt, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hga_status hga_route_groups(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                            const void* group_sum, int64_t t_cap, const int32_t* chunk_idx,
+                            const int32_t* chunk_cnt, int32_t* group_idx, int32_t* group_cnt,
+                            hga_stream_t stream) {
+  return route_common(p, q, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+                      group_cnt, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                      const void* k, const void* v, int64_t t_cap, const int32_t* group_idx,
+                      const int32_t* group_cnt, void* o, float* lse, hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!q || !k || !v || !group_idx || !group_cnt || !o) return HGA_ERR_INVALID_ARG;
+  hga::AttendArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q_start = q_start;
+  a.n_q = n_q;
+  a.t_cap = t_cap;
+  a.group_idx = group_idx;
+  a.group_cnt = group_cnt;
+  a.cap_g = cap_groups(p, t_cap);
+  a.o = o;
+  a.lse = lse;
+  a.n_blocks = (int)((n_q + p->qblock - 1) / p->qblock);
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.G = p->n_q_heads / p->n_kv_heads;
+  a.group = p->group;
+  a.qblock = p->qblock;
+  a.sink = p->sink;
+  a.local = p->local;
+  const int64_t max_list = p->sink / p->group + a.cap_g + p->local / p->group +
+                           (p->qblock + p->group - 1) / p->group;
+  if (max_list > 16384) return HGA_ERR_UNSUPPORTED;
+  a.max_list = (int)max_list;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->head_dim));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? launch_attend_bf16<128>(a, st) : launch_attend_bf16<64>(a, st);
+  return p->head_dim == 128 ? launch_attend_f32<128>(a, st) : launch_attend_f32<64>(a, st);
+}
+
+hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                       const void* k, const void* v, int64_t t_cap, void* chunk_sum,
+                       void* group_sum, int32_t* chunk_idx, int32_t* chunk_cnt,
+                       int32_t* group_idx, int32_t* group_cnt, void* o, float* lse,
+                       hga_stream_t stream) {
+  hga_status s = hga_build_summaries(p, k, t_cap, q_start, q_start + n_q, chunk_sum, group_sum,
+                                     stream);
+  if (s != HGA_OK) return s;
+  s = hga_route_chunks(p, q, q_start, n_q, chunk_sum, t_cap, chunk_idx, chunk_cnt, stream);
+  if (s != HGA_OK) return s;
+  s = hga_route_groups(p, q, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+                       group_cnt, stream);
+  if (s != HGA_OK) return s;
+  return hga_attend(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
+}
+
+hga_status hga_check(hga_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return HGA_ERR_CUDA;
+  int st = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&st, hga::g_status, sizeof(int)) != cudaSuccess) return HGA_ERR_CUDA;
+  if (st != 0 && cudaMemcpyToSymbol(hga::g_status, &zero, sizeof(int)) != cudaSuccess)
+    return HGA_ERR_CUDA;
+  return (hga_status)st;
+}
+
+const char* hga_status_string(hga_status s) {
+  switch (s) {
+    case HGA_OK: return "HGA_OK";
+    case HGA_ERR_INVALID_ARG: return "HGA_ERR_INVALID_ARG";
+    case HGA_ERR_UNSUPPORTED: return "HGA_ERR_UNSUPPORTED";
+    case HGA_ERR_CUDA: return "HGA_ERR_CUDA";
+    case HGA_ERR_DEVICE_CHECK: return "HGA_ERR_DEVICE_CHECK";
+    case HGA_ERR_TIMEOUT: return "HGA_ERR_TIMEOUT";
+  }
+  return "HGA_ERR_UNKNOWN";
+}
+
+int64_t hga_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

@@ -1,0 +1,221 @@
+"""ctypes binding of libhga.so (argument marshalling only).
+
+Every step of the routed-attention path runs in the library's CUDA kernels;
+this module only turns torch tensors into pointers and sizes, picks the
+current CUDA stream and maps status codes to exceptions.  There is no Python
+or CPU fallback: if libhga.so cannot be loaded, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhga.so")
+
+HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED = 0, 1, 2
+HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK, HGA_ERR_TIMEOUT = 3, 4, 5
+HGA_BF16, HGA_FP32 = 0, 1
+
+EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
+            "hga_attend", "hga_forward", "hga_index_capacity",
+            "hga_validate_params", "hga_check", "hga_status_string",
+            "hga_launch_count")
+
+
+class HgaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)}")
+
+
+class CParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_q_heads", "n_kv_heads", "head_dim", "chunk", "group", "qblock",
+        "sink", "local", "top_chunks", "top_groups", "dtype")]
+
+
+@dataclasses.dataclass(frozen=True)
+class Params:
+    """Mirror of the C struct hga_params."""
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    chunk: int = 64
+    group: int = 8
+    qblock: int = 64
+    sink: int = 64
+    local: int = 128
+    top_chunks: int = 4
+    top_groups: int = 8
+    dtype: str = "bf16"
+
+    def c(self) -> CParams:
+        return CParams(self.n_q_heads, self.n_kv_heads, self.head_dim,
+                       self.chunk, self.group, self.qblock, self.sink,
+                       self.local, self.top_chunks, self.top_groups,
+                       HGA_BF16 if self.dtype == "bf16" else HGA_FP32)
+
+    @property
+    def torch_dtype(self):
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    @staticmethod
+    def from_workload(w) -> "Params":
+        return Params(w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.group,
+                      w.qblock, w.sink, w.local, w.top_chunks, w.top_groups,
+                      w.dtype)
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m long_context_hga_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(CParams)
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    sig = {
+        "hga_build_summaries": [P, vp, i64, i64, i64, vp, vp, vp],
+        "hga_route_chunks": [P, vp, i64, i64, vp, i64, vp, vp, vp],
+        "hga_route_groups": [P, vp, i64, i64, vp, i64, vp, vp, vp, vp, vp],
+        "hga_attend": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp],
+        "hga_forward": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp,
+                        vp, vp, vp],
+        "hga_index_capacity": [P, i64, i32],
+        "hga_validate_params": [P],
+        "hga_check": [vp],
+        "hga_status_string": [ctypes.c_int],
+        "hga_launch_count": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.hga_index_capacity.restype = ctypes.c_int64
+    lib.hga_launch_count.restype = ctypes.c_int64
+    lib.hga_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+LIB = _load()
+
+
+def status_string(code: int) -> str:
+    return LIB.hga_status_string(code).decode()
+
+
+def _ok(code: int, what: str):
+    if code != HGA_OK:
+        raise HgaError(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libhga must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def validate_params(p: Params) -> int:
+    return LIB.hga_validate_params(ctypes.byref(p.c()))
+
+
+def index_capacity(p: Params, t_cap: int, which: int) -> int:
+    return LIB.hga_index_capacity(ctypes.byref(p.c()), t_cap, which)
+
+
+def launch_count() -> int:
+    return LIB.hga_launch_count()
+
+
+def check(stream=None) -> int:
+    """Synchronise and return (and clear) the device status word."""
+    return LIB.hga_check(_stream(stream))
+
+
+def build_summaries(p: Params, k, t_begin: int, t_end: int, chunk_sum,
+                    group_sum, stream=None):
+    t_cap = k.shape[1]
+    _ok(LIB.hga_build_summaries(ctypes.byref(p.c()), _ptr(k), t_cap, t_begin,
+                                t_end, _ptr(chunk_sum), _ptr(group_sum),
+                                _stream(stream)), "hga_build_summaries")
+
+
+def route_chunks(p: Params, q, q_start: int, chunk_sum, t_cap: int,
+                 chunk_idx, chunk_cnt, stream=None):
+    _ok(LIB.hga_route_chunks(ctypes.byref(p.c()), _ptr(q), q_start, q.shape[0],
+                             _ptr(chunk_sum), t_cap, _ptr(chunk_idx),
+                             _ptr(chunk_cnt), _stream(stream)),
+        "hga_route_chunks")
+
+
+def route_groups(p: Params, q, q_start: int, group_sum, t_cap: int, chunk_idx,
+                 chunk_cnt, group_idx, group_cnt, stream=None):
+    _ok(LIB.hga_route_groups(ctypes.byref(p.c()), _ptr(q), q_start, q.shape[0],
+                             _ptr(group_sum), t_cap, _ptr(chunk_idx),
+                             _ptr(chunk_cnt), _ptr(group_idx), _ptr(group_cnt),
+                             _stream(stream)), "hga_route_groups")
+
+
+def attend(p: Params, q, q_start: int, k, v, group_idx, group_cnt, o,
+           lse=None, stream=None):
+    _ok(LIB.hga_attend(ctypes.byref(p.c()), _ptr(q), q_start, q.shape[0],
+                       _ptr(k), _ptr(v), k.shape[1], _ptr(group_idx),
+                       _ptr(group_cnt), _ptr(o), _ptr(lse), _stream(stream)),
+        "hga_attend")
+
+
+def forward(p: Params, q, q_start: int, k, v, bufs: "Buffers", stream=None):
+    _ok(LIB.hga_forward(ctypes.byref(p.c()), _ptr(q), q_start, q.shape[0],
+                        _ptr(k), _ptr(v), k.shape[1], _ptr(bufs.chunk_sum),
+                        _ptr(bufs.group_sum), _ptr(bufs.chunk_idx),
+                        _ptr(bufs.chunk_cnt), _ptr(bufs.group_idx),
+                        _ptr(bufs.group_cnt), _ptr(bufs.o), _ptr(bufs.lse),
+                        _stream(stream)), "hga_forward")
+
+
+@dataclasses.dataclass
+class Buffers:
+    """Device buffers of one routed-attention problem (allocated by torch)."""
+    chunk_sum: torch.Tensor
+    group_sum: torch.Tensor
+    chunk_idx: torch.Tensor
+    chunk_cnt: torch.Tensor
+    group_idx: torch.Tensor
+    group_cnt: torch.Tensor
+    o: torch.Tensor
+    lse: Optional[torch.Tensor]
+
+
+def allocate(p: Params, t_cap: int, n_q: int, device="cuda",
+             with_lse: bool = True) -> Buffers:
+    d, Hkv = p.head_dim, p.n_kv_heads
+    nb = (n_q + p.qblock - 1) // p.qblock
+    cc, cg = index_capacity(p, t_cap, 0), index_capacity(p, t_cap, 1)
+    if cc < 0 or cg < 0:
+        raise HgaError(HGA_ERR_INVALID_ARG, "index_capacity")
+    dt = p.torch_dtype
+    i32 = torch.int32
+    return Buffers(
+        chunk_sum=torch.zeros(Hkv, t_cap // p.chunk, d, dtype=dt, device=device),
+        group_sum=torch.zeros(Hkv, t_cap // p.group, d, dtype=dt, device=device),
+        chunk_idx=torch.empty(Hkv, nb, max(cc, 1), dtype=i32, device=device),
+        chunk_cnt=torch.empty(Hkv, nb, dtype=i32, device=device),
+        group_idx=torch.empty(Hkv, nb, max(cg, 1), dtype=i32, device=device),
+        group_cnt=torch.empty(Hkv, nb, dtype=i32, device=device),
+        o=torch.empty(n_q, p.n_q_heads, d, dtype=dt, device=device),
+        lse=torch.empty(n_q, p.n_q_heads, dtype=torch.float32, device=device)
+        if with_lse else None,
+    )

@@ -1,0 +1,145 @@
+"""CUDA path vs CPU oracle through the C ABI (needs a B200).
+
+Small sizes compare every (query block, KV head) unit; the full-size
+workloads run in the same launch configuration as bench.py and compare
+sampled units.  Ragged tails (a last query block shorter than 64) and the
+first blocks (sink, local and diagonal overlapping) are covered.
+"""
+import numpy as np
+import pytest
+import torch
+
+import hga_inputs as gi
+from oracle import hga_oracle as ho
+import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(w, units=None, split_history=True, t_cap=None):
+    inp = gi.make_inputs(w)
+    g = parity.run_gpu(w, inp, t_cap=t_cap, split_history=split_history)
+    rep = parity.compare(w, inp, g, units=units)
+    print(w.name, rep)
+    assert rep.ok(), rep
+    return rep, g, inp
+
+
+def test_tiny_fp32_all_units():
+    _check(gi.TINY_FP32)
+
+
+def test_tiny_fp32_ragged_and_capacity():
+    # context not a multiple of 64, t_cap larger than the context
+    _check(gi.TINY_FP32.with_(T=1000), t_cap=1088)
+
+
+def test_qwen3_8b_shape_reduced_ragged():
+    _check(gi.QWEN3_8B_16K.with_(T=2088, n_needles=8), split_history=False)
+
+
+def test_qwen3_30b_shape_reduced_ragged():
+    _check(gi.QWEN3_30B_64K.with_(T=8168, q0=6144, n_needles=16))
+
+
+def test_head_dim_64_bf16_no_gqa():
+    w = gi.Workload("d64_g1", 4, 4, 64, 1536, 512, 1e6, 64, 128, 3, 10,
+                    n_needles=4)
+    _check(w)
+
+
+def test_gqa16_rows_span_slices():
+    # 16 query heads per KV head: 1024 rows per block, several row slices
+    w = gi.Workload("g16", 16, 1, 128, 1600, 1024, 1e6, 128, 128, 5, 12,
+                    n_needles=4)
+    _check(w)
+
+
+def test_budget_covers_everything_is_dense():
+    """Full budget must reproduce dense causal attention."""
+    w = gi.SWEEP_32K.with_(T=1280, top_chunks=0, top_groups=0, n_needles=4)
+    rep, g, inp = _check(w)
+    q, k, v = gi.to_f64(inp.q), gi.to_f64(inp.k), gi.to_f64(inp.v)
+    Od, Ld = ho.dense_causal_attention(q, k, v, w.q0, w.n_q_heads)
+    atol, rtol = parity.TOL["bf16"]
+    assert (np.abs(g.o - Od) <= atol + rtol * np.abs(Od)).all()
+    assert abs(rep.density - 1.0) < 1e-12
+
+
+@pytest.mark.parametrize("kc", [4, 8, 16, 64, 0])
+def test_budget_sweep_reduced(kc):
+    w = gi.SWEEP_32K.with_(T=4096, top_chunks=kc,
+                           top_groups=2 * kc if kc > 0 else 0, n_needles=8)
+    units = parity.sample_units(w, 40)
+    _check(w, units=units)
+
+
+def test_exact_ties_go_to_lower_index():
+    """Identical chunk summaries give exactly equal scores on both sides;
+    the lower chunk / group index must win."""
+    w = gi.Workload("ties", 8, 2, 128, 2048, 1536, 1e6, 64, 128, 5, 7)
+    inp = gi.make_inputs(w)
+    k = inp.k.clone()
+    base = k[:, 64:128].clone()
+    for c in range(1, 1536 // 64):      # every candidate chunk identical
+        k[:, 64 * c:64 * (c + 1)] = base
+    inp = gi.Inputs(w, inp.q, k, inp.v, [])
+    g = parity.run_gpu(w, inp)
+    for h in range(2):
+        for b in range(8):
+            ch = list(g.chunk_idx[h, b, :g.chunk_cnt[h, b]])
+            assert ch == [1, 2, 3, 4, 5], ch
+    rep = parity.compare(w, inp, g)
+    assert rep.chunk_mismatch == 0 and rep.invalid_choice == 0
+
+
+def test_empty_and_tiny_segments():
+    from long_context_hga_b200 import hga
+    w = gi.TINY_FP32.with_(dtype="bf16", T=64)
+    p = hga.Params.from_workload(w)
+    dev = "cuda:0"
+    bufs = hga.allocate(p, 64, 0, device=dev)
+    k = torch.zeros(1, 64, 64, dtype=torch.bfloat16, device=dev)
+    q = torch.zeros(0, 2, 64, dtype=torch.bfloat16, device=dev)
+    n0 = hga.launch_count()
+    hga.forward(p, q, 0, k, k, bufs)            # n_q = 0: nothing launched
+    assert hga.launch_count() == n0
+    for T in (1, 7, 8, 63, 65):
+        _check(gi.TINY_FP32.with_(T=T, dtype="bf16"), t_cap=128)
+
+
+def test_bad_group_index_sets_device_status():
+    """Out-of-range routed groups are skipped and reported, never read."""
+    from long_context_hga_b200 import hga
+    w = gi.TINY_FP32.with_(dtype="bf16")
+    inp = gi.make_inputs(w)
+    p = hga.Params.from_workload(w)
+    dev = "cuda:0"
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    hga.forward(p, q, 0, k, v, bufs)
+    assert hga.check() == 0
+    gi_bad = bufs.group_idx.clone()
+    gi_bad[0, -1, 0] = 10 ** 6          # far outside the context
+    gi_bad[0, -2, 0] = gi_bad[0, -2, 1]  # duplicate -> not ascending
+    o2 = torch.empty_like(bufs.o)
+    hga.attend(p, q, 0, k, v, gi_bad, bufs.group_cnt, o2)
+    assert hga.check() == hga.HGA_ERR_DEVICE_CHECK
+    assert hga.check() == 0             # cleared
+    assert torch.isfinite(o2.float()).all()
+    ci_bad = bufs.chunk_idx.clone()
+    ci_bad[0, -1, 0] = -5
+    hga.route_groups(p, q, 0, bufs.group_sum, w.T, ci_bad, bufs.chunk_cnt,
+                     bufs.group_idx, bufs.group_cnt)
+    assert hga.check() == hga.HGA_ERR_DEVICE_CHECK
+
+
+@pytest.mark.parametrize("name", ["qwen3_30b_a3b_64k_last2k",
+                                  "qwen3_8b_prefill_16k"])
+def test_full_size_sampled(name):
+    """Full-size workloads in the benchmark's launch configuration; the
+    oracle recomputes a sample of units."""
+    w = gi.WORKLOADS[name]
+    units = parity.sample_units(w, 12)
+    rep, _, _ = _check(w, units=units)
+    assert rep.compared_units >= 10
