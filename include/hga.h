@@ -175,6 +175,10 @@ const char* hga_status_string(hga_status s);
  * accounting in benchmarks); never reset. */
 int64_t hga_launch_count(void);
 
+/* Text of the last CUDA error seen by this thread inside the library (the
+ * cause behind an HGA_ERR_CUDA); static storage, never NULL. */
+const char* hga_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -73,6 +73,27 @@ __device__ __forceinline__ int build_group_list(const AttendArgs& a, int b, int 
   return n;
 }
 
+// Converts n16 16-byte chunks of bf16 at `tile` (shared memory) to fp16 in
+// place, cooperatively over `nthreads` threads.  bf16 -> fp16 is exact for
+// 2^-14 <= |x| < 65504 (8 significant bits fit in 11) and loses at most 2^-25
+// below; a finite value that overflows fp16 is reported (HGA_ERR_DEVICE_CHECK).
+__device__ __forceinline__ void convert_tile_bf16_to_f16(char* tile, int n16, int nthreads) {
+  bool overflow = false;
+  for (int i = threadIdx.x; i < n16; i += nthreads) {
+    uint4 raw = *reinterpret_cast<const uint4*>(tile + i * 16);
+    uint32_t* w = reinterpret_cast<uint32_t*>(&raw);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      overflow |= (fabsf(f.x) > 65504.f) | (fabsf(f.y) > 65504.f);
+      __half2 hv = __floats2half2_rn(f.x, f.y);
+      w[j] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    *reinterpret_cast<uint4*>(tile + i * 16) = raw;
+  }
+  if (overflow) report(HGA_ERR_DEVICE_CHECK);
+}
+
 // ---------------------------------------------------------------- bf16, mma.sync
 
 constexpr int kAttRows = 64;      // rows per CTA (4 warps x 16)
@@ -164,6 +185,8 @@ __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
     }
     const char* tk = sk + (t & 1) * (kAttTok * D * 2);
     const char* tv = sv + (t & 1) * (kAttTok * D * 2);
+    // V tile bf16 -> fp16 in place (exact for |v| < 65504; larger is reported)
+    convert_tile_bf16_to_f16(sv + (t & 1) * (kAttTok * D * 2), kAttTok * D / 8, 128);
     float s[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -224,8 +247,8 @@ __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
       const float p3 = exp2f(s[nt][3] * a.scale_log2 - use_b);
       sum_a += p0 + p1;
       sum_b += p2 + p3;
-      __nv_bfloat162 lo = __floats2bfloat162_rn(p0, p1);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(p2, p3);
+      __half2 lo = __floats2half2_rn(p0, p1);
+      __half2 hi = __floats2half2_rn(p2, p3);
       pf[nt >> 1][(nt & 1) * 2 + 0] = *reinterpret_cast<uint32_t*>(&lo);
       pf[nt >> 1][(nt & 1) * 2 + 1] = *reinterpret_cast<uint32_t*>(&hi);
     }
@@ -238,7 +261,10 @@ __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
       oacc[nd][2] *= corr_b;
       oacc[nd][3] *= corr_b;
     }
-    // O += P V   (A = P from registers: a0 = rows g / tokens 2t of n-tile 2kk, ...)
+    // O += P V in fp16 x fp16 -> fp32 (A = P from registers: a0 = rows g /
+    // tokens 2t of n-tile 2kk, ...).  P in [0, 1] keeps 11 significant bits in
+    // fp16 against 8 in bf16.
+    __syncthreads();   // converted V tile visible
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       uint32_t af[4] = {pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3]};
@@ -248,8 +274,8 @@ __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
         const int ch = nd2 * 2 + (lane >> 4);
         uint32_t v0, v1, v2, v3;
         ldsm_x4_t(smem_u32(tv + swz<D>(r, ch)), v0, v1, v2, v3);
-        mma_bf16(oacc[2 * nd2], af, v0, v1);
-        mma_bf16(oacc[2 * nd2 + 1], af, v2, v3);
+        mma_f16(oacc[2 * nd2], af, v0, v1);
+        mma_f16(oacc[2 * nd2 + 1], af, v2, v3);
       }
     }
     __syncthreads();

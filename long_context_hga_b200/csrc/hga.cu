@@ -14,29 +14,43 @@
 namespace {
 
 std::atomic<int64_t> g_launches{0};
+thread_local cudaError_t g_last_cuda = cudaSuccess;
 
-inline hga_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? HGA_OK : HGA_ERR_CUDA; }
+inline hga_status cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return HGA_OK;
+  g_last_cuda = e;
+  return HGA_ERR_CUDA;
+}
 
 inline hga_status after_launch() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cuda_ok(cudaGetLastError());
 }
 
-// Opt every kernel into the full 227 KB of dynamic shared memory once per
-// device (the attribute is per device context).
+// Opt every kernel into all the dynamic shared memory a block may use (227 KB
+// minus the kernel's static shared memory), once per device (the attribute
+// belongs to the device context).
+constexpr size_t kMaxSmemPerBlock = 227 * 1024;
+
 template <auto kernel>
 hga_status allow_smem(size_t bytes) {
   static std::atomic<uint64_t> done{0};
+  static std::atomic<size_t> dyn_max{0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return HGA_ERR_CUDA;
-  if (bytes > 227 * 1024) return HGA_ERR_UNSUPPORTED;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_ok(e);
   const uint64_t bit = 1ull << (dev & 63);
-  if (done.load(std::memory_order_acquire) & bit) return HGA_OK;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-      cudaSuccess)
-    return HGA_ERR_CUDA;
-  done.fetch_or(bit, std::memory_order_acq_rel);
-  return HGA_OK;
+  if (!(done.load(std::memory_order_acquire) & bit)) {
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kernel)) != cudaSuccess) return cuda_ok(e);
+    const size_t avail = kMaxSmemPerBlock - fa.sharedSizeBytes;
+    if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)avail)) != cudaSuccess)
+      return cuda_ok(e);
+    dyn_max.store(avail, std::memory_order_relaxed);
+    done.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  return bytes <= dyn_max.load(std::memory_order_relaxed) ? HGA_OK : HGA_ERR_UNSUPPORTED;
 }
 
 hga_status check_params(const hga_params* p) {
@@ -142,12 +156,13 @@ hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_beg
   const int64_t c_last = (t_end + chunk - 1) / chunk;   // partial chunk: its closed groups
   const int64_t n_chunks = c_last - c_first;
   if (n_chunks <= 0) return HGA_OK;
-  const int64_t warps = (int64_t)Hkv * n_chunks;
-  const int64_t blocks = (warps + 7) / 8;
-  if (blocks > 0x7fffffff) return HGA_ERR_UNSUPPORTED;
-  hga::summaries_kernel<T, D><<<(unsigned)blocks, 256, 0, st>>>(
-      reinterpret_cast<const T*>(k), t_cap, Hkv, c_first, n_chunks, t_end, chunk, group,
-      reinterpret_cast<T*>(cs), reinterpret_cast<T*>(gs));
+  if (n_chunks > 0x7fffffff || Hkv > 65535) return HGA_ERR_UNSUPPORTED;
+  (void)chunk;
+  (void)group;   // 64 / 8, validated by check_params
+  dim3 grid((unsigned)n_chunks, Hkv);
+  hga::summaries_kernel<T, D><<<grid, 32 * hga::kSumGroupsPerChunk, 0, st>>>(
+      reinterpret_cast<const T*>(k), t_cap, c_first, t_end, reinterpret_cast<T*>(cs),
+      reinterpret_cast<T*>(gs));
   return after_launch();
 }
 
@@ -279,12 +294,12 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start, int6
 }
 
 hga_status hga_check(hga_stream_t stream) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return HGA_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_ok(e);
   int st = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&st, hga::g_status, sizeof(int)) != cudaSuccess) return HGA_ERR_CUDA;
-  if (st != 0 && cudaMemcpyToSymbol(hga::g_status, &zero, sizeof(int)) != cudaSuccess)
-    return HGA_ERR_CUDA;
+  if ((e = cudaMemcpyFromSymbol(&st, hga::g_status, sizeof(int))) != cudaSuccess) return cuda_ok(e);
+  if (st != 0 && (e = cudaMemcpyToSymbol(hga::g_status, &zero, sizeof(int))) != cudaSuccess)
+    return cuda_ok(e);
   return (hga_status)st;
 }
 
@@ -301,5 +316,7 @@ const char* hga_status_string(hga_status s) {
 }
 
 int64_t hga_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* hga_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 
 }  // extern "C"

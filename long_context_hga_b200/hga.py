@@ -24,7 +24,7 @@ HGA_BF16, HGA_FP32 = 0, 1
 EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_attend", "hga_forward", "hga_index_capacity",
             "hga_validate_params", "hga_check", "hga_status_string",
-            "hga_launch_count")
+            "hga_launch_count", "hga_last_cuda_error")
 
 
 class HgaError(RuntimeError):
@@ -91,6 +91,7 @@ def _load() -> ctypes.CDLL:
         "hga_check": [vp],
         "hga_status_string": [ctypes.c_int],
         "hga_launch_count": [],
+        "hga_last_cuda_error": [],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -99,6 +100,7 @@ def _load() -> ctypes.CDLL:
     lib.hga_index_capacity.restype = ctypes.c_int64
     lib.hga_launch_count.restype = ctypes.c_int64
     lib.hga_status_string.restype = ctypes.c_char_p
+    lib.hga_last_cuda_error.restype = ctypes.c_char_p
     return lib
 
 
@@ -110,6 +112,8 @@ def status_string(code: int) -> str:
 
 
 def _ok(code: int, what: str):
+    if code == HGA_ERR_CUDA:
+        raise HgaError(code, f"{what} ({LIB.hga_last_cuda_error().decode()})")
     if code != HGA_OK:
         raise HgaError(code, what)
 

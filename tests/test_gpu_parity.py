@@ -81,7 +81,7 @@ def test_exact_ties_go_to_lower_index():
     inp = gi.make_inputs(w)
     k = inp.k.clone()
     base = k[:, 64:128].clone()
-    for c in range(1, 1536 // 64):      # every candidate chunk identical
+    for c in range(1, 2048 // 64):      # every candidate chunk identical
         k[:, 64 * c:64 * (c + 1)] = base
     inp = gi.Inputs(w, inp.q, k, inp.v, [])
     g = parity.run_gpu(w, inp)
