@@ -179,6 +179,17 @@ int64_t hga_launch_count(void);
  * cause behind an HGA_ERR_CUDA); static storage, never NULL. */
 const char* hga_last_cuda_error(void);
 
+/* Diagnostic switch (process-wide) of the bf16 kernels behind hga_attend,
+ * hga_route_chunks, hga_route_groups and hga_forward: 0 = automatic (the
+ * tcgen05 tensor-core kernels whenever the shapes allow them: 16-byte aligned
+ * operands; attention: 128 divisible by the query heads per KV head and at
+ * most 4608 attended groups per block; routing: at most 8 query heads per KV
+ * head and 4096 candidates per block), 1 = the portable mma.sync kernels,
+ * 2 = same as 0.  Both variants compute the same function; tests use the
+ * switch to check one against the other.  Returns HGA_ERR_INVALID_ARG for any
+ * other value. */
+hga_status hga_set_kernel_variant(int32_t variant);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,492 @@
+// Step 4 on the sm_100a tensor cores: gathered exact-token attention with
+// tcgen05.mma, TMEM accumulators and TMA gathers of the routed groups.
+//
+// "Long-Context Fine-Tuning with Limited VRAM", section 2.1: exact token K/V
+// of the kept groups plus the sink and local windows feed softmax attention.
+//
+// One CTA = 256 query rows of one (query block, KV head) unit, as two 128-row
+// tiles Q0/Q1 (rows are (position, query head) pairs, so the G heads that
+// share the KV head reuse every gathered K/V tile).  K/V arrive in 128-token
+// tiles (16 routed 8-token groups); each group is one contiguous 8 x d span of
+// the head-major cache and is fetched by TMA as 8-row x 128-byte boxes with
+// the 128-byte swizzle, which is exactly one swizzle atom of the tcgen05
+// operand layout, so arbitrary group lists need no repacking.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
+//   warp 1      TMEM owner and MMA issuer (one thread):
+//                 S_i = Q_i K^T   (bf16 x bf16 -> fp32, K-major A and B)
+//                 O_i += P_i V    (fp16 P from TMEM x fp16 V, MN-major B)
+//   warps 2-3   convert each V tile bf16 -> fp16 in place (exact below 65504;
+//               P kept in fp16 has 11 significant bits) and zero rows that
+//               hold no attended token
+//   warps 4-7   softmax of tile Q0, warps 8-11 softmax of tile Q1: one thread
+//               per row reads its S row from TMEM, applies the causal / padding
+//               mask, keeps the running max and sum in fp32, writes P (fp16)
+//               over its S columns and rescales O only when the max grows by
+//               more than 2^8 (exact: O and the sum always share one max)
+// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D).
+// While one softmax warpgroup works, the MMA warp runs the other tile's
+// products, so the tensor pipe and the exponentials overlap.
+#pragma once
+#include "attend.cuh"
+#include "tc.cuh"
+
+namespace hga {
+
+constexpr int kTcRows = 128;              // rows per Q tile (MMA M)
+constexpr int kTcTok = 128;               // tokens per K/V tile (MMA N of S)
+constexpr int kTcGroupsPerTile = kTcTok / 8;
+constexpr int kTcThreads = 384;
+constexpr int kTcSlots = 4;               // K/V ring: one K or V tile per slot
+constexpr int kTcMaxList = 4608;          // group-list slots in shared memory
+constexpr float kTcRescaleLog2 = 8.0f;
+
+struct TcArgs {
+  AttendArgs a;
+  int rows_per_cta;                       // 256
+};
+
+template <int D>
+struct TcLayout {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kHalfBytes = kTcRows * 128;                 // 16 KB
+  static constexpr int kQBytes = 2 * kHalves * kHalfBytes;         // 2 tiles
+  static constexpr int kGroupBytes = kHalves * 8 * 128;            // one 8-token group
+  static constexpr int kSlotBytes = kTcGroupsPerTile * kGroupBytes;  // one K or V tile
+  static constexpr int kQOff = 0;
+  static constexpr int kSlotOff = kQOff + kQBytes;
+  static constexpr int kBarOff = kSlotOff + kTcSlots * kSlotBytes;
+  static constexpr int kListOff = kBarOff + 512;
+  static constexpr size_t smem_bytes(int max_list) {
+    return 1024 + (size_t)kListOff + (size_t)max_list * 4;
+  }
+};
+
+struct TcBars {
+  uint64_t q_full, full[kTcSlots], empty[kTcSlots], v_ready[kTcSlots];
+  uint64_t s_full[2], p_full[2], o_full[2], done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+#ifdef HGA_TIMELINE
+// Debug build only: globaltimer stamps of pipeline events of CTA (0,0,0).
+__device__ unsigned long long g_tl[8192];
+__device__ unsigned int g_tl_n;
+__device__ __forceinline__ void tl_mark(int kind, int idx) {
+  if (blockIdx.x | blockIdx.y | blockIdx.z) return;
+  const unsigned int k = atomicAdd(&g_tl_n, 1u);
+  if (k < 8192) g_tl[k] = (tc::globaltimer_ns() << 16) | ((unsigned)kind << 10) | (unsigned)(idx & 1023);
+}
+#define HGA_TL(kind, idx) tl_mark(kind, idx)
+#else
+#define HGA_TL(kind, idx) ((void)0)
+#endif
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k1,
+                     const __grid_constant__ CUtensorMap tm_k8,
+                     const __grid_constant__ CUtensorMap tm_v1,
+                     const __grid_constant__ CUtensorMap tm_v8, TcArgs args) {
+  using L = TcLayout<D>;
+  const AttendArgs& a = args.a;
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* smem = reinterpret_cast<char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  TcBars* bars = reinterpret_cast<TcBars*>(smem + L::kBarOff);
+  int* list = reinterpret_cast<int*>(smem + L::kListOff);
+  volatile int* abort_flag = &bars->abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.y, h = blockIdx.z;
+  const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
+  const int64_t T = a.q_start + a.n_q;
+  const int npos = (int)min((int64_t)a.qblock, T - b0);
+  const int nrows = npos * a.G;
+  const int row0 = blockIdx.x * args.rows_per_cta;     // first unit row of this CTA
+  if (row0 >= nrows) return;
+  const int nq = (nrows - row0) > kTcRows ? 2 : 1;     // Q tiles with live rows
+
+  // ---- prologue: group list, barriers, TMEM
+  int n_nondiag;
+  bool inv = false;
+  if (tid == 0) bars->abort = 0;
+  const int n_list = build_group_list(a, b, h, b0, T, list, &n_nondiag, &inv);
+  if (n_list < 0) return;                       // uniform; reported inside
+  __shared__ int s_inv;
+  if (tid == 0) s_inv = 0;
+  __syncthreads();
+  if (inv) s_inv = 1;
+  if (tid == 0) {
+    tc::mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < kTcSlots; ++s) {
+      tc::mbar_init(&bars->full[s], 1);
+      tc::mbar_init(&bars->empty[s], 1);
+      tc::mbar_init(&bars->v_ready[s], 64);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bars->s_full[i], 1);
+      tc::mbar_init(&bars->p_full[i], kTcRows);
+      tc::mbar_init(&bars->o_full[i], 1);
+    }
+    tc::mbar_init(&bars->done, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+  const bool any_invalid = s_inv != 0;
+  const int n_tiles = (n_list + kTcGroupsPerTile - 1) / kTcGroupsPerTile;
+  const int n_loads = 2 * n_tiles;             // K0 V0 K1 V1 ... through the ring
+
+  char* sQ = smem + L::kQOff;
+  auto slot_ptr = [&](int s, int half) {
+    return smem + L::kSlotOff + s * L::kSlotBytes + half * 1024;
+  };
+
+  if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = tc::idesc_f16(kTcRows, kTcTok, 1, 0);
+      constexpr uint32_t kIdPV = tc::idesc_f16(kTcRows, D, 0, 1);
+      const uint32_t q_base = tc::smem_addr(sQ);
+      bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
+      tc::fence_after_sync();
+      auto issue_s = [&](int i, int s) {
+        for (int k = 0; k < D / 16; ++k) {
+          const int hf = k >> 2, kk = k & 3;
+          const uint64_t ad = tc::sdesc_sw128(
+              q_base + (i * L::kHalves + hf) * L::kHalfBytes + kk * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(tc::smem_addr(slot_ptr(s, 0)) + hf * 1024 + kk * 32, 16,
+                                              L::kGroupBytes);
+          tc::mma_ss(tmem + i * 128, ad, bd, kIdS, k > 0);
+        }
+        tc::mma_commit(&bars->s_full[i]);
+      };
+      auto issue_pv = [&](int i, int s, bool first) {
+        for (int k = 0; k < kTcTok / 16; ++k) {
+          const uint64_t bd =
+              tc::sdesc_sw128(tc::smem_addr(slot_ptr(s, 0)) + 2 * k * L::kGroupBytes, 1024,
+                              L::kGroupBytes);
+          tc::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, bd, kIdPV, (!first) || k > 0);
+        }
+        tc::mma_commit(&bars->o_full[i]);
+      };
+      // PV of tile jp for every Q tile, then release V_jp's slot
+      auto pv_all = [&](int jp) -> bool {
+        const int nv = 2 * jp + 1, sv = nv % kTcSlots;
+        if (!tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag)) return false;
+        for (int i = 0; i < nq; ++i) {
+          if (!tc::mbar_wait(&bars->p_full[i], jp & 1, abort_flag)) return false;
+          tc::fence_after_sync();
+          issue_pv(i, sv, jp == 0);
+          HGA_TL(3, jp * 2 + i);
+        }
+        tc::mma_commit(&bars->empty[sv]);
+        return true;
+      };
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int nk = 2 * j, sk = nk % kTcSlots;
+        if (!(ok = tc::mbar_wait(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
+        tc::fence_after_sync();
+        if (j > 0) {
+          // Q tile 0: PV(j-1) then S(j); Q tile 1 likewise, so each softmax
+          // warpgroup finds its next S while the other tile's products run
+          const int nv = 2 * (j - 1) + 1, sv = nv % kTcSlots;
+          if (!(ok = tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag))) break;
+          for (int i = 0; i < nq && ok; ++i) {
+            if (!(ok = tc::mbar_wait(&bars->p_full[i], (j - 1) & 1, abort_flag))) break;
+            tc::fence_after_sync();
+            issue_pv(i, sv, j - 1 == 0);
+            HGA_TL(3, (j - 1) * 2 + i);
+            issue_s(i, sk);
+            HGA_TL(2, j * 2 + i);
+          }
+          if (!ok) break;
+          tc::mma_commit(&bars->empty[sv]);
+        } else {
+          for (int i = 0; i < nq; ++i) {
+            issue_s(i, sk);
+            HGA_TL(2, i);
+          }
+        }
+        tc::mma_commit(&bars->empty[sk]);
+      }
+      if (ok && n_tiles > 0) ok = pv_all(n_tiles - 1);
+      // drain: every MMA issued so far has completed before TMEM is freed
+      tc::mma_commit(&bars->done);
+      const uint64_t t0 = tc::globaltimer_ns();
+      while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    // Load n of the ring is K_{n/2} (n even) or V_{n/2} (n odd), into slot
+    // n % kTcSlots.  A slot holds 16 groups as [group][half][8 rows][128 B]
+    // (2 KB per group, 128-byte swizzle), which is what one box of the 4-D
+    // tensor view (64 dims, 8 rows, 2 halves, group) lands as; 8 aligned
+    // consecutive groups (sink, local window, diagonal, adjacent routed
+    // groups) come in one 16 KB box.  Lane e < 16 owns entry e of the tile.
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tm_q);
+      tc::tma_prefetch_desc(&tm_k1);
+      tc::tma_prefetch_desc(&tm_k8);
+      tc::tma_prefetch_desc(&tm_v1);
+      tc::tma_prefetch_desc(&tm_v8);
+      tc::mbar_arrive_expect_tx(&bars->q_full, nq * L::kHalves * L::kHalfBytes);
+    }
+    __syncwarp();
+    if (lane < nq * L::kHalves) {
+      const int i = lane / L::kHalves, hf = lane % L::kHalves;
+      const int pos0 = (int)(b0 - a.q_start) + row0 / a.G;
+      tc::tma_load_3d(sQ + (i * L::kHalves + hf) * L::kHalfBytes, &tm_q, hf * 64, h * a.G,
+                      pos0 + i * (kTcRows / a.G), &bars->q_full);
+    }
+    int last_use[kTcSlots];
+#pragma unroll
+    for (int s = 0; s < kTcSlots; ++s) last_use[s] = -1;
+    const int e = lane & 15;
+    const int64_t head_group0 = (int64_t)h * (a.t_cap / a.group);
+    for (int n = 0; n < n_loads; ++n) {
+      const int s = n % kTcSlots, u = n / kTcSlots, j = n >> 1;
+      int ok = 1;
+      if (n >= kTcSlots && lane == 0) ok = tc::mbar_wait(&bars->empty[s], (u - 1) & 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      const int li = j * kTcGroupsPerTile + e;
+      const int ent = li < n_list ? list[li] : -1;
+      // runs: entries 8r..8r+7 are 8 consecutive valid groups
+      const int ent0 = __shfl_sync(0xffffffffu, ent, e & ~7);
+      const bool consec = ent >= 0 && ent0 >= 0 && ent == ent0 + (e & 7);
+      const unsigned cons_mask = __ballot_sync(0xffffffffu, lane < 16 && consec);
+      const bool run = ((cons_mask >> (e & ~7)) & 0xffu) == 0xffu;
+      const unsigned valid = __ballot_sync(0xffffffffu, lane < 16 && ent >= 0);
+      if (lane == 0)
+        tc::mbar_arrive_expect_tx(&bars->full[s], __popc(valid) * L::kHalves * 1024);
+      __syncwarp();
+      if (lane < 16 && ent >= 0) {
+        const bool vt = n & 1;
+        const int gcoord = (int)(head_group0 + ent);
+        if (run) {
+          if ((e & 7) == 0)
+            tc::tma_load_4d(slot_ptr(s, 0) + e * L::kGroupBytes, vt ? &tm_v8 : &tm_k8, 0, 0, 0,
+                            gcoord, &bars->full[s]);
+        } else {
+          tc::tma_load_4d(slot_ptr(s, 0) + e * L::kGroupBytes, vt ? &tm_v1 : &tm_k1, 0, 0, 0,
+                          gcoord, &bars->full[s]);
+        }
+      }
+      last_use[s] = u;
+      if (lane == 0) HGA_TL(1, n);
+    }
+    // make sure no copy is still landing in shared memory when we leave
+    if (lane == 0) {
+      for (int s = 0; s < kTcSlots; ++s) {
+        if (last_use[s] < 0) continue;
+        const uint64_t t0 = tc::globaltimer_ns();
+        while (!tc::mbar_try_wait(&bars->full[s], last_use[s] & 1) &&
+               tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ V converter
+    // bf16 -> fp16 in place (exact below 65504; a larger magnitude is
+    // reported), then rows that hold no attended token (padding entries,
+    // tokens past the context) are zeroed so that P = 0 meets finite V.
+    const int ct = tid - 64;   // 0..63
+    constexpr int kChunks = L::kSlotBytes / 16;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int nv = 2 * j + 1, s = nv % kTcSlots;
+      if (!tc::mbar_wait(&bars->full[s], (nv / kTcSlots) & 1, abort_flag)) break;
+      if (ct == 0) HGA_TL(4, j);
+      const int li0 = j * kTcGroupsPerTile;
+      bool clean = li0 + kTcGroupsPerTile <= n_list && !any_invalid;
+      if (clean) clean = ((int64_t)list[li0 + kTcGroupsPerTile - 1] + 1) * a.group <= T;
+      char* base = slot_ptr(s, 0);
+      uint32_t vmax = 0;
+#pragma unroll 4
+      for (int q = ct; q < kChunks; q += 64) {
+        bool live = true;
+        if (!clean) {
+          // offset -> (group, row): [group][half][8 rows][128 B]; rows that
+          // were not loaded hold stale bytes and are only zeroed
+          const int g = (q * 16) / L::kGroupBytes;
+          const int rr = ((q * 16) % 1024) / 128;
+          const int li = li0 + g;
+          const int ent = li < n_list ? list[li] : -1;
+          live = ent >= 0 && (int64_t)ent * a.group + rr < T;
+        }
+        uint4 raw = make_uint4(0, 0, 0, 0);
+        if (live) {
+          raw = *reinterpret_cast<const uint4*>(base + q * 16);
+          uint32_t* w = reinterpret_cast<uint32_t*>(&raw);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            vmax = __vmaxu2(vmax, w[t] & 0x7fff7fffu);
+            w[t] = tc::pack_half2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xffff0000u));
+          }
+        }
+        *reinterpret_cast<uint4*>(base + q * 16) = raw;
+      }
+      if ((vmax & 0xffffu) >= 0x4780u || (vmax >> 16) >= 0x4780u) report(HGA_ERR_DEVICE_CHECK);
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars->v_ready[s]);
+      if (ct == 0) HGA_TL(7, j);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int i = (warp - 4) >> 2;              // Q tile of this warpgroup
+    const int quarter = warp & 3;               // TMEM lane quarter
+    const int r = quarter * 32 + lane;          // row within the Q tile
+    const int unit_row = row0 + i * kTcRows + r;
+    const bool row_live = (i < nq) && unit_row < nrows;
+    const int64_t pos = b0 + (row_live ? unit_row / a.G : 0);
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + i * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + i * 128;
+    float m = -INFINITY, l = 0.f;
+    bool ok = i < nq;
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      if (!(ok = tc::mbar_wait(&bars->s_full[i], j & 1, abort_flag))) break;
+      if (tid == 128 || tid == 256) HGA_TL(5, j * 2 + i);
+      tc::fence_after_sync();
+      // S row in two 64-column halves (bounded register use): pass 1 finds
+      // the row max, pass 2 turns the same columns into P.
+      const bool need_mask = any_invalid || (j * kTcGroupsPerTile + kTcGroupsPerTile > n_nondiag);
+      uint32_t sr[64];
+      auto load_half = [&](int hf) {
+        tc::tmem_ld32(t_s + hf * 64, sr);
+        tc::tmem_ld32(t_s + hf * 64 + 32, sr + 32);
+        tc::tmem_wait_ld();
+        if (need_mask) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int li = j * kTcGroupsPerTile + hf * 8 + e;
+            const int ent = li < n_list ? list[li] : -1;
+            const int64_t tok0 = (int64_t)ent * a.group;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              if (ent < 0 || tok0 + c > pos) sr[e * 8 + c] = __float_as_uint(-INFINITY);
+          }
+        }
+      };
+      // 8 independent partial maxima (no 128-long dependency chain)
+      float mx8[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        load_half(hf);
+#pragma unroll
+        for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      }
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      mx *= a.scale_log2;
+      const float m_new = fmaxf(m, mx);
+      float m_use = m, corr = 1.f;
+      bool rescale = false;
+      if (m == -INFINITY) {
+        // nothing accumulated yet (O and l are zero): start at this tile's
+        // max; a row with no valid token yet keeps -inf and gets p = 0
+        m_use = m_new == -INFINITY ? 0.f : m_new;
+        m = m_new;
+        corr = 0.f;
+      } else if (m_new - m > kTcRescaleLog2) {
+        m_use = m_new;
+        corr = tc::ex2(m - m_new);
+        rescale = true;
+        m = m_new;
+      }
+      if (__any_sync(0xffffffffu, rescale) && j > 0) {
+        // O holds PV of tiles < j: wait for the last one, then scale in TMEM
+        if (!(ok = tc::mbar_wait(&bars->o_full[i], (j - 1) & 1, abort_flag))) break;
+        tc::fence_after_sync();
+        const float f = rescale ? corr : 1.f;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tc::tmem_ld32(t_o + c * 32, orr);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * f);
+          tc::tmem_st32(t_o + c * 32, orr);
+        }
+        tc::tmem_wait_st();
+      }
+      l *= corr;
+      const float neg = -m_use;
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+#pragma unroll 1
+      for (int hf = 0; hf < 2; ++hf) {
+        load_half(hf);
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = tc::ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, neg));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, neg));
+          rs4[(c >> 1) & 3] += p0 + p1;
+          pk[c >> 1] = tc::pack_half2(p0, p1);
+        }
+        // fp16 P of tokens [64hf, 64hf+64) -> columns [32hf, 32hf+32): those
+        // S columns were consumed by pass 1 and by this half's reload
+        tc::tmem_st32(t_s + hf * 32, pk);
+      }
+      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
+      tc::tmem_wait_st();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&bars->p_full[i]);
+      if (tid == 128 || tid == 256) HGA_TL(6, j * 2 + i);
+    }
+    // ---- epilogue: O / l -> bf16, LSE
+    if (ok && i < nq && n_tiles > 0 && tc::mbar_wait(&bars->o_full[i], (n_tiles - 1) & 1, abort_flag)) {
+      tc::fence_after_sync();
+      const float inv_l = 1.f / l;
+      __nv_bfloat16* dst = nullptr;
+      if (row_live)
+        dst = reinterpret_cast<__nv_bfloat16*>(a.o) +
+              ((pos - a.q_start) * a.Hq + (int64_t)h * a.G + unit_row % a.G) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        tc::tmem_ld32(t_o + c * 32, orr);
+        tc::tmem_wait_ld();
+        if (row_live) {
+#pragma unroll
+          for (int q = 0; q < 32; q += 8) {
+            uint4 pk4;
+            uint32_t* pw = reinterpret_cast<uint32_t*>(&pk4);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[q + 2 * t]) * inv_l,
+                                                        __uint_as_float(orr[q + 2 * t + 1]) * inv_l);
+              pw[t] = *reinterpret_cast<uint32_t*>(&v2);
+            }
+            *reinterpret_cast<uint4*>(dst + c * 32 + q) = pk4;
+          }
+        }
+      }
+      if (row_live && a.lse)
+        a.lse[(pos - a.q_start) * a.Hq + (int64_t)h * a.G + unit_row % a.G] =
+            (m + log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  // ---- teardown: all roles done (every wait above is bounded)
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace hga

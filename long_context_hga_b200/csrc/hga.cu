@@ -2,6 +2,9 @@
 // checks, launch sizing and the device status word; the kernels live in the
 // included .cuh files.  One translation unit so that the status word is a
 // single device symbol without relocatable device code.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <atomic>
 #include <cstdio>
 
@@ -10,6 +13,8 @@
 #include "summaries.cuh"
 #include "route.cuh"
 #include "attend.cuh"
+#include "attend_tc.cuh"
+#include "route_tc.cuh"
 
 namespace {
 
@@ -82,6 +87,70 @@ hga_status check_segment(const hga_params* p, int64_t q_start, int64_t n_q, int6
   return HGA_OK;
 }
 
+// ---------------------------------------------------------------- TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> fn{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  f = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  fn.store(f, std::memory_order_release);
+  return f;
+}
+
+// bf16 tensor map with the 128-byte swizzle; dims/box innermost first,
+// strides in bytes for dims 1..rank-1.  Out-of-range elements read as zero.
+bool encode_bf16_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides, const uint32_t* box) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base),
+             reinterpret_cast<const cuuint64_t*>(dims), reinterpret_cast<const cuuint64_t*>(strides),
+             reinterpret_cast<const cuuint32_t*>(box), estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 0 = choose, 1 = portable mma.sync kernels, 2 = tcgen05 kernels (when eligible)
+std::atomic<int> g_kernel_variant{0};
+
+// ---------------------------------------------------------------- routing
+
+bool route_tc_eligible(const hga::RouteArgs& a, const void* q, const void* summ) {
+  const uintptr_t align = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(summ);
+  return (align & 15) == 0 && (a.G == 1 || a.G == 2 || a.G == 4 || a.G == 8) &&
+         a.max_cands <= hga::kRtMaxCands && (int64_t)a.Hkv * a.n_summ_cap < (1ll << 31) &&
+         a.n_q < (1ll << 31);
+}
+
+template <int D>
+hga_status launch_route_tc(hga::RouteArgs& a, cudaStream_t st) {
+  using L = hga::RtLayout<D>;
+  hga_status s = allow_smem<hga::route_tc_kernel<D>>(L::kSmem);
+  if (s != HGA_OK) return s;
+  hga::RtArgs ra{a, std::min(256, 64 * a.G)};
+  CUtensorMap tq, ts, ts8;
+  const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
+  const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)a.Hq * D * 2};
+  const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(ra.rs / a.G)};
+  const uint64_t sd[2] = {(uint64_t)D, (uint64_t)a.Hkv * a.n_summ_cap};
+  const uint64_t ss[1] = {(uint64_t)D * 2};
+  const uint32_t sb[2] = {64, (uint32_t)hga::kRtTile};
+  const uint32_t sb8[2] = {64, 8};
+  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb) || !encode_bf16_map(&ts, a.summ, 2, sd, ss, sb) ||
+      !encode_bf16_map(&ts8, a.summ, 2, sd, ss, sb8))
+    return HGA_ERR_CUDA;
+  dim3 grid(a.n_blocks, a.Hkv);
+  hga::route_tc_kernel<D><<<grid, hga::kRtThreads, L::kSmem, st>>>(tq, ts, ts8, ra);
+  return after_launch();
+}
+
 constexpr int kMaxRouteCands = 16384;
 constexpr int kMaxKeptChunks = 2048;
 
@@ -143,9 +212,12 @@ hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int
     if (a.in_cap > kMaxKeptChunks || a.in_cap * per > kMaxRouteCands) return HGA_ERR_UNSUPPORTED;
     a.max_cands = (int)std::max<int64_t>(a.in_cap * per, 1);
   }
-  if (p->dtype == HGA_BF16)
+  if (p->dtype == HGA_BF16) {
+    if (g_kernel_variant.load(std::memory_order_relaxed) != 1 && route_tc_eligible(a, q, summ))
+      return p->head_dim == 128 ? launch_route_tc<128>(a, st) : launch_route_tc<64>(a, st);
     return p->head_dim == 128 ? launch_route<__nv_bfloat16, 128>(a, st)
                               : launch_route<__nv_bfloat16, 64>(a, st);
+  }
   return p->head_dim == 128 ? launch_route<float, 128>(a, st) : launch_route<float, 64>(a, st);
 }
 
@@ -167,7 +239,43 @@ hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_beg
 }
 
 template <int D>
+hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
+  using L = hga::TcLayout<D>;
+  const size_t smem = L::smem_bytes(a.max_list);
+  hga_status s = allow_smem<hga::attend_tc_kernel<D>>(smem);
+  if (s != HGA_OK) return s;
+  CUtensorMap tq, tk1, tk8, tv1, tv8;
+  const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
+  const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)a.Hq * D * 2};
+  const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(hga::kTcRows / a.G)};
+  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb)) return HGA_ERR_CUDA;
+  // K/V as (64 dims, 8 rows, D/64 halves, group): one box = whole groups
+  // landing as [group][half][8 rows][128 B]
+  const uint64_t gd[4] = {64, 8, (uint64_t)(D / 64), (uint64_t)a.Hkv * a.t_cap / 8};
+  const uint64_t gs[3] = {(uint64_t)D * 2, 128, (uint64_t)D * 2 * 8};
+  const uint32_t b1[4] = {64, 8, (uint32_t)(D / 64), 1};
+  const uint32_t b8[4] = {64, 8, (uint32_t)(D / 64), 8};
+  if (!encode_bf16_map(&tk1, a.k, 4, gd, gs, b1) || !encode_bf16_map(&tk8, a.k, 4, gd, gs, b8) ||
+      !encode_bf16_map(&tv1, a.v, 4, gd, gs, b1) || !encode_bf16_map(&tv8, a.v, 4, gd, gs, b8))
+    return HGA_ERR_CUDA;
+  hga::TcArgs ta{a, 2 * hga::kTcRows};
+  dim3 grid((a.qblock * a.G + ta.rows_per_cta - 1) / ta.rows_per_cta, a.n_blocks, a.Hkv);
+  hga::attend_tc_kernel<D><<<grid, hga::kTcThreads, smem, st>>>(tq, tk1, tk8, tv1, tv8, ta);
+  return after_launch();
+}
+
+bool tc_eligible(const hga::AttendArgs& a) {
+  const uintptr_t align = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
+                          reinterpret_cast<uintptr_t>(a.v);
+  return (align & 15) == 0 && a.G <= hga::kTcRows && (hga::kTcRows % a.G) == 0 &&
+         a.max_list <= hga::kTcMaxList && (int64_t)a.Hkv * a.t_cap < (1ll << 31) &&
+         a.n_q < (1ll << 31) && (a.t_cap % a.group) == 0;
+}
+
+template <int D>
 hga_status launch_attend_bf16(hga::AttendArgs& a, cudaStream_t st) {
+  const int variant = g_kernel_variant.load(std::memory_order_relaxed);
+  if (variant != 1 && tc_eligible(a)) return launch_attend_tc<D>(a, st);
   const size_t smem = hga::attend_mma_smem_bytes<D>(a.max_list);
   hga_status s = allow_smem<hga::attend_mma_kernel<D>>(smem);
   if (s != HGA_OK) return s;
@@ -316,6 +424,27 @@ const char* hga_status_string(hga_status s) {
 }
 
 int64_t hga_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+#ifdef HGA_TIMELINE
+// Debug builds only (not part of the ABI): copies the attention kernel's
+// event stamps of CTA (0,0,0) and resets them; returns the count.
+int hga_debug_timeline(unsigned long long* out, int max) {
+  unsigned int n = 0, zero = 0;
+  cudaDeviceSynchronize();
+  cudaMemcpyFromSymbol(&n, hga::g_tl_n, sizeof(n));
+  if (n > 8192) n = 8192;
+  if ((int)n > max) n = (unsigned)max;
+  cudaMemcpyFromSymbol(out, hga::g_tl, n * sizeof(unsigned long long));
+  cudaMemcpyToSymbol(hga::g_tl_n, &zero, sizeof(zero));
+  return (int)n;
+}
+#endif
+
+hga_status hga_set_kernel_variant(int32_t variant) {
+  if (variant < 0 || variant > 2) return HGA_ERR_INVALID_ARG;
+  g_kernel_variant.store(variant, std::memory_order_relaxed);
+  return HGA_OK;
+}
 
 const char* hga_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 

@@ -24,7 +24,8 @@ HGA_BF16, HGA_FP32 = 0, 1
 EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_attend", "hga_forward", "hga_index_capacity",
             "hga_validate_params", "hga_check", "hga_status_string",
-            "hga_launch_count", "hga_last_cuda_error")
+            "hga_launch_count", "hga_last_cuda_error",
+            "hga_set_kernel_variant")
 
 
 class HgaError(RuntimeError):
@@ -92,6 +93,7 @@ def _load() -> ctypes.CDLL:
         "hga_status_string": [ctypes.c_int],
         "hga_launch_count": [],
         "hga_last_cuda_error": [],
+        "hga_set_kernel_variant": [i32],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -223,3 +225,8 @@ def allocate(p: Params, t_cap: int, n_q: int, device="cuda",
         lse=torch.empty(n_q, p.n_q_heads, dtype=torch.float32, device=device)
         if with_lse else None,
     )
+
+
+def set_kernel_variant(variant: int):
+    """0 = automatic (tcgen05 kernel when eligible), 1 = portable mma.sync."""
+    _ok(LIB.hga_set_kernel_variant(variant), "hga_set_kernel_variant")

@@ -143,3 +143,15 @@ def test_full_size_sampled(name):
     units = parity.sample_units(w, 12)
     rep, _, _ = _check(w, units=units)
     assert rep.compared_units >= 10
+
+
+@pytest.mark.parametrize("variant", [1, 0])
+def test_attend_variants_agree_with_oracle(variant):
+    """Both bf16 attention kernels (portable mma.sync and tcgen05) pass the
+    same parity check, with a ragged tail and GQA 8."""
+    from long_context_hga_b200 import hga
+    hga.set_kernel_variant(variant)
+    try:
+        _check(gi.QWEN3_30B_64K.with_(T=4136, q0=2048, n_needles=8))
+    finally:
+        hga.set_kernel_variant(0)
