@@ -179,6 +179,13 @@ int64_t hga_launch_count(void);
  * cause behind an HGA_ERR_CUDA); static storage, never NULL. */
 const char* hga_last_cuda_error(void);
 
+/* Self-test of the software 2^x the attention kernel evaluates on the FMA
+ * pipe for part of each softmax row (Cody-Waite reduction + degree-4
+ * polynomial, relative error below 3e-6 for -125 <= x <= 127; smaller x
+ * gives 2^-125).  Device arrays x, y of n floats; y[i] = 2^x[i].  Not part of
+ * the method: it lets a test compare the kernel's exponential with exp2f. */
+hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t stream);
+
 /* Diagnostic switch (process-wide) of the bf16 kernels behind hga_attend,
  * hga_route_chunks, hga_route_groups and hga_forward: 0 = automatic (the
  * tcgen05 tensor-core kernels whenever the shapes allow them: 16-byte aligned

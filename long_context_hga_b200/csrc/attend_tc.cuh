@@ -71,15 +71,26 @@ struct TcBars {
 };
 
 #ifdef HGA_TIMELINE
-// Debug build only: globaltimer stamps of pipeline events of CTA (0,0,0).
+// Debug builds only: SM clock stamps of pipeline events of CTA (0,0,0), kept
+// in shared memory (one region per role, no global round trips while the
+// kernel runs) and copied out at exit.
 __device__ unsigned long long g_tl[8192];
 __device__ unsigned int g_tl_n;
-__device__ __forceinline__ void tl_mark(int kind, int idx) {
+__device__ unsigned long long g_cta[3 * 4096];   // per CTA: start ns, end ns, SM id
+struct TlBuf {
+  unsigned long long ev[5][128];
+  unsigned int n[5];
+  long long t0;
+};
+__device__ __forceinline__ void tl_mark(TlBuf* bf, int kind, int idx) {
   if (blockIdx.x | blockIdx.y | blockIdx.z) return;
-  const unsigned int k = atomicAdd(&g_tl_n, 1u);
-  if (k < 8192) g_tl[k] = (tc::globaltimer_ns() << 16) | ((unsigned)kind << 10) | (unsigned)(idx & 1023);
+  const int r = kind == 1 ? 0 : (kind <= 3 ? 1 : (kind == 4 || kind == 7 ? 2 : (threadIdx.x < 256 ? 3 : 4)));
+  const unsigned int k = atomicAdd(&bf->n[r], 1u);
+  if (k < 128)
+    bf->ev[r][k] = ((unsigned long long)(clock64() - bf->t0) << 16) | ((unsigned)kind << 10) |
+                   (unsigned)(idx & 1023);
 }
-#define HGA_TL(kind, idx) tl_mark(kind, idx)
+#define HGA_TL(kind, idx) tl_mark(&s_tl, kind, idx)
 #else
 #define HGA_TL(kind, idx) ((void)0)
 #endif
@@ -118,6 +129,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (n_list < 0) return;                       // uniform; reported inside
   __shared__ int s_inv;
   if (tid == 0) s_inv = 0;
+#ifdef HGA_TIMELINE
+  __shared__ TlBuf s_tl;
+  if (tid < 5) s_tl.n[tid] = 0;
+  if (tid == 0) s_tl.t0 = clock64();
+  const int cta_lin = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  if (tid == 0 && cta_lin < 4096) {
+    unsigned int smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_cta[3 * cta_lin] = tc::globaltimer_ns();
+    g_cta[3 * cta_lin + 2] = smid;
+  }
+#endif
   __syncthreads();
   if (inv) s_inv = 1;
   if (tid == 0) {
@@ -160,24 +183,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t q_base = tc::smem_addr(sQ);
       bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
       tc::fence_after_sync();
+      // Descriptors are built once; a k-step only moves the start-address
+      // field (bytes >> 4, compile-time offsets), so the issue loop is a
+      // handful of integer adds per MMA and keeps the tensor pipe fed.
+      const uint64_t q_desc0 = tc::sdesc_sw128(q_base, 16, 1024);
+      const uint64_t slot_desc0 = tc::sdesc_sw128(tc::smem_addr(slot_ptr(0, 0)), 16, L::kGroupBytes);
+      const uint64_t v_desc0 = tc::sdesc_sw128(tc::smem_addr(slot_ptr(0, 0)), 1024, L::kGroupBytes);
       auto issue_s = [&](int i, int s) {
+        const uint64_t ad = q_desc0 + (uint64_t)((i * L::kHalves * L::kHalfBytes) >> 4);
+        const uint64_t bd = slot_desc0 + (uint64_t)((s * L::kSlotBytes) >> 4);
+#pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const int hf = k >> 2, kk = k & 3;
-          const uint64_t ad = tc::sdesc_sw128(
-              q_base + (i * L::kHalves + hf) * L::kHalfBytes + kk * 32, 16, 1024);
-          const uint64_t bd = tc::sdesc_sw128(tc::smem_addr(slot_ptr(s, 0)) + hf * 1024 + kk * 32, 16,
-                                              L::kGroupBytes);
-          tc::mma_ss(tmem + i * 128, ad, bd, kIdS, k > 0);
+          constexpr int unused = 0;
+          (void)unused;
+          tc::mma_ss(tmem + i * 128, ad + (uint64_t)((((k >> 2) * L::kHalfBytes) + (k & 3) * 32) >> 4),
+                     bd + (uint64_t)((((k >> 2) * 1024) + (k & 3) * 32) >> 4), kIdS, k > 0);
         }
         tc::mma_commit(&bars->s_full[i]);
       };
       auto issue_pv = [&](int i, int s, bool first) {
-        for (int k = 0; k < kTcTok / 16; ++k) {
-          const uint64_t bd =
-              tc::sdesc_sw128(tc::smem_addr(slot_ptr(s, 0)) + 2 * k * L::kGroupBytes, 1024,
-                              L::kGroupBytes);
-          tc::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8, bd, kIdPV, (!first) || k > 0);
-        }
+        const uint64_t bd = v_desc0 + (uint64_t)((s * L::kSlotBytes) >> 4);
+        const uint32_t acc0 = first ? 0u : 1u;
+#pragma unroll
+        for (int k = 0; k < kTcTok / 16; ++k)
+          tc::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
+                     bd + (uint64_t)((2 * k * L::kGroupBytes) >> 4), kIdPV, k > 0 ? 1u : acc0);
         tc::mma_commit(&bars->o_full[i]);
       };
       // PV of tile jp for every Q tile, then release V_jp's slot
@@ -195,29 +225,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       };
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int nk = 2 * j, sk = nk % kTcSlots;
-        if (!(ok = tc::mbar_wait(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
-        tc::fence_after_sync();
-        if (j > 0) {
-          // Q tile 0: PV(j-1) then S(j); Q tile 1 likewise, so each softmax
-          // warpgroup finds its next S while the other tile's products run
-          const int nv = 2 * (j - 1) + 1, sv = nv % kTcSlots;
-          if (!(ok = tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag))) break;
-          for (int i = 0; i < nq && ok; ++i) {
+        const int nv = 2 * (j - 1) + 1, sv = nv % kTcSlots;
+        if (j > 0 && !(ok = tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag)))
+          break;
+        // Per Q tile: PV(j-1) (needs only P(j-1) and V(j-1)), then S(j)
+        // (needs K(j)); each softmax warpgroup finds its next S while the
+        // other tile's products run.
+        for (int i = 0; i < nq && ok; ++i) {
+          if (j > 0) {
             if (!(ok = tc::mbar_wait(&bars->p_full[i], (j - 1) & 1, abort_flag))) break;
             tc::fence_after_sync();
             issue_pv(i, sv, j - 1 == 0);
             HGA_TL(3, (j - 1) * 2 + i);
-            issue_s(i, sk);
-            HGA_TL(2, j * 2 + i);
           }
-          if (!ok) break;
-          tc::mma_commit(&bars->empty[sv]);
-        } else {
-          for (int i = 0; i < nq; ++i) {
-            issue_s(i, sk);
-            HGA_TL(2, i);
+          if (i == 0) {
+            if (!(ok = tc::mbar_wait(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
+            tc::fence_after_sync();
           }
+          issue_s(i, sk);
+          HGA_TL(2, j * 2 + i);
         }
+        if (!ok) break;
+        if (j > 0) tc::mma_commit(&bars->empty[sv]);
         tc::mma_commit(&bars->empty[sk]);
       }
       if (ok && n_tiles > 0) ok = pv_all(n_tiles - 1);
@@ -298,11 +327,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ V converter
-    // bf16 -> fp16 in place (exact below 65504; a larger magnitude is
-    // reported), then rows that hold no attended token (padding entries,
-    // tokens past the context) are zeroed so that P = 0 meets finite V.
+    // bf16 -> fp16 in place (exact below 65504; a larger magnitude becomes
+    // inf and is caught by the epilogue's finite check), then rows that hold
+    // no attended token (padding entries, tokens past the context) are
+    // zeroed so that P = 0 always meets finite V.
     const int ct = tid - 64;   // 0..63
     constexpr int kChunks = L::kSlotBytes / 16;
+    auto cvt4 = [](uint4& r) {
+      uint32_t* w = reinterpret_cast<uint32_t*>(&r);
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        w[t] = tc::pack_half2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xffff0000u));
+    };
     for (int j = 0; j < n_tiles; ++j) {
       const int nv = 2 * j + 1, s = nv % kTcSlots;
       if (!tc::mbar_wait(&bars->full[s], (nv / kTcSlots) & 1, abort_flag)) break;
@@ -311,32 +347,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool clean = li0 + kTcGroupsPerTile <= n_list && !any_invalid;
       if (clean) clean = ((int64_t)list[li0 + kTcGroupsPerTile - 1] + 1) * a.group <= T;
       char* base = slot_ptr(s, 0);
-      uint32_t vmax = 0;
-#pragma unroll 4
-      for (int q = ct; q < kChunks; q += 64) {
-        bool live = true;
-        if (!clean) {
+      if (clean) {
+#pragma unroll
+        for (int q0 = 0; q0 < kChunks; q0 += 64 * 8) {
+          uint4 raw[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) raw[x] = *reinterpret_cast<const uint4*>(base + (q0 + x * 64 + ct) * 16);
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            cvt4(raw[x]);
+            *reinterpret_cast<uint4*>(base + (q0 + x * 64 + ct) * 16) = raw[x];
+          }
+        }
+      } else {
+        for (int q = ct; q < kChunks; q += 64) {
           // offset -> (group, row): [group][half][8 rows][128 B]; rows that
           // were not loaded hold stale bytes and are only zeroed
           const int g = (q * 16) / L::kGroupBytes;
           const int rr = ((q * 16) % 1024) / 128;
           const int li = li0 + g;
           const int ent = li < n_list ? list[li] : -1;
-          live = ent >= 0 && (int64_t)ent * a.group + rr < T;
-        }
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (live) {
-          raw = *reinterpret_cast<const uint4*>(base + q * 16);
-          uint32_t* w = reinterpret_cast<uint32_t*>(&raw);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            vmax = __vmaxu2(vmax, w[t] & 0x7fff7fffu);
-            w[t] = tc::pack_half2(__uint_as_float(w[t] << 16), __uint_as_float(w[t] & 0xffff0000u));
+          uint4 raw = make_uint4(0, 0, 0, 0);
+          if (ent >= 0 && (int64_t)ent * a.group + rr < T) {
+            raw = *reinterpret_cast<const uint4*>(base + q * 16);
+            cvt4(raw);
           }
+          *reinterpret_cast<uint4*>(base + q * 16) = raw;
         }
-        *reinterpret_cast<uint4*>(base + q * 16) = raw;
       }
-      if ((vmax & 0xffffu) >= 0x4780u || (vmax >> 16) >= 0x4780u) report(HGA_ERR_DEVICE_CHECK);
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars->v_ready[s]);
       if (ct == 0) HGA_TL(7, j);
@@ -358,36 +396,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!(ok = tc::mbar_wait(&bars->s_full[i], j & 1, abort_flag))) break;
       if (tid == 128 || tid == 256) HGA_TL(5, j * 2 + i);
       tc::fence_after_sync();
-      // S row in two 64-column halves (bounded register use): pass 1 finds
-      // the row max, pass 2 turns the same columns into P.
+      // The whole S row (128 columns) is read from TMEM once, masked,
+      // reduced to its max, then turned into P in place.
       const bool need_mask = any_invalid || (j * kTcGroupsPerTile + kTcGroupsPerTile > n_nondiag);
-      uint32_t sr[64];
-      auto load_half = [&](int hf) {
-        tc::tmem_ld32(t_s + hf * 64, sr);
-        tc::tmem_ld32(t_s + hf * 64 + 32, sr + 32);
-        tc::tmem_wait_ld();
-        if (need_mask) {
+      uint32_t sr[kTcTok];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int li = j * kTcGroupsPerTile + hf * 8 + e;
-            const int ent = li < n_list ? list[li] : -1;
-            const int64_t tok0 = (int64_t)ent * a.group;
+      for (int c = 0; c < kTcTok / 32; ++c) tc::tmem_ld32(t_s + c * 32, sr + c * 32);
+      tc::tmem_wait_ld();
+      if (need_mask) {
+        // token indices fit in 32 bits on this path (Hkv * t_cap < 2^31)
+        const int pos32 = (int)pos;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              if (ent < 0 || tok0 + c > pos) sr[e * 8 + c] = __float_as_uint(-INFINITY);
-          }
+        for (int e = 0; e < kTcGroupsPerTile; ++e) {
+          const int li = j * kTcGroupsPerTile + e;
+          const int ent = li < n_list ? list[li] : -1;
+          const int lim = ent < 0 ? -1 : pos32 - ent * 8;   // valid columns c <= lim
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            if (c > lim) sr[e * 8 + c] = __float_as_uint(-INFINITY);
         }
-      };
+      }
       // 8 independent partial maxima (no 128-long dependency chain)
       float mx8[8];
 #pragma unroll
       for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        load_half(hf);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-      }
+      for (int c = 0; c < kTcTok; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= a.scale_log2;
@@ -406,8 +440,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         rescale = true;
         m = m_new;
       }
+      l *= corr;
+      const float neg = -m_use;
+      // p = 2^(s*scale - m) in packed pairs: 6 of every 16 columns on the
+      // FMA pipe (exp2_fma2), the rest on the MUFU unit, so neither unit
+      // alone limits the row; sums in two packed accumulators.
+      const uint64_t scale2 = tc::pk2(a.scale_log2, a.scale_log2);
+      const uint64_t neg2 = tc::pk2(neg, neg);
+      uint64_t sum2[2] = {tc::pk2(0.f, 0.f), tc::pk2(0.f, 0.f)};
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const uint64_t x2 = tc::ffma2(tc::pk2(__uint_as_float(sr[64 * hf + c]),
+                                                __uint_as_float(sr[64 * hf + c + 1])),
+                                       scale2, neg2);
+          uint64_t p2;
+          if (((c >> 1) & 7) >= 5) {
+            p2 = tc::exp2_fma2(x2);
+          } else {
+            float x0, x1;
+            tc::unpk2(x2, x0, x1);
+            p2 = tc::pk2(tc::ex2(x0), tc::ex2(x1));
+          }
+          sum2[(c >> 1) & 1] = tc::fadd2(sum2[(c >> 1) & 1], p2);
+          float p0, p1;
+          tc::unpk2(p2, p0, p1);
+          pk[c >> 1] = tc::pack_half2(p0, p1);
+        }
+        // fp16 P of tokens [64hf, 64hf+64) -> columns [32hf, 32hf+32) (the
+        // whole S row is already in registers)
+        tc::tmem_st32(t_s + hf * 32, pk);
+      }
+      {
+        float a0, a1, b0v, b1v;
+        tc::unpk2(sum2[0], a0, a1);
+        tc::unpk2(sum2[1], b0v, b1v);
+        l += (a0 + a1) + (b0v + b1v);
+      }
       if (__any_sync(0xffffffffu, rescale) && j > 0) {
-        // O holds PV of tiles < j: wait for the last one, then scale in TMEM
+        // O holds PV of tiles < j (PV of tile j waits for p_full below):
+        // wait for the last one, then scale O in TMEM.  Done after P so the
+        // S row's registers are free.
         if (!(ok = tc::mbar_wait(&bars->o_full[i], (j - 1) & 1, abort_flag))) break;
         tc::fence_after_sync();
         const float f = rescale ? corr : 1.f;
@@ -420,27 +495,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int q = 0; q < 32; ++q) orr[q] = __float_as_uint(__uint_as_float(orr[q]) * f);
           tc::tmem_st32(t_o + c * 32, orr);
         }
-        tc::tmem_wait_st();
       }
-      l *= corr;
-      const float neg = -m_use;
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        load_half(hf);
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = tc::ex2(fmaf(__uint_as_float(sr[c]), a.scale_log2, neg));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(sr[c + 1]), a.scale_log2, neg));
-          rs4[(c >> 1) & 3] += p0 + p1;
-          pk[c >> 1] = tc::pack_half2(p0, p1);
-        }
-        // fp16 P of tokens [64hf, 64hf+64) -> columns [32hf, 32hf+32): those
-        // S columns were consumed by pass 1 and by this half's reload
-        tc::tmem_st32(t_s + hf * 32, pk);
-      }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->p_full[i]);
@@ -449,7 +504,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---- epilogue: O / l -> bf16, LSE
     if (ok && i < nq && n_tiles > 0 && tc::mbar_wait(&bars->o_full[i], (n_tiles - 1) & 1, abort_flag)) {
       tc::fence_after_sync();
+      if (tid == 128 || tid == 256) HGA_TL(8, i);
       const float inv_l = 1.f / l;
+      bool nonfinite = false;   // inf/NaN output: V outside the fp16 range (or bad input)
       __nv_bfloat16* dst = nullptr;
       if (row_live)
         dst = reinterpret_cast<__nv_bfloat16*>(a.o) +
@@ -466,8 +523,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t* pw = reinterpret_cast<uint32_t*>(&pk4);
 #pragma unroll
             for (int t = 0; t < 4; ++t) {
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(orr[q + 2 * t]) * inv_l,
-                                                        __uint_as_float(orr[q + 2 * t + 1]) * inv_l);
+              const float o0 = __uint_as_float(orr[q + 2 * t]) * inv_l;
+              const float o1 = __uint_as_float(orr[q + 2 * t + 1]) * inv_l;
+              nonfinite |= !(fabsf(o0) <= 3.0e38f) | !(fabsf(o1) <= 3.0e38f);
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
               pw[t] = *reinterpret_cast<uint32_t*>(&v2);
             }
             *reinterpret_cast<uint4*>(dst + c * 32 + q) = pk4;
@@ -477,6 +536,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (row_live && a.lse)
         a.lse[(pos - a.q_start) * a.Hq + (int64_t)h * a.G + unit_row % a.G] =
             (m + log2f(l)) * 0.6931471805599453f;
+      if (row_live && nonfinite) report(HGA_ERR_DEVICE_CHECK);
+      if (tid == 128 || tid == 256) HGA_TL(9, i);
     }
   }
 
@@ -487,6 +548,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
+#ifdef HGA_TIMELINE
+  if (tid == 0 && cta_lin < 4096) g_cta[3 * cta_lin + 1] = tc::globaltimer_ns();
+  if (tid == 0 && !(blockIdx.x | blockIdx.y | blockIdx.z)) {
+    unsigned int k = 0;
+    for (int r = 0; r < 5; ++r)
+      for (unsigned int x = 0; x < min(s_tl.n[r], 128u) && k < 8192; ++x) g_tl[k++] = s_tl.ev[r][x];
+    g_tl_n = k;
+  }
+#endif
 }
 
 }  // namespace hga

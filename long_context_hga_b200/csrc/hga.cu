@@ -438,7 +438,28 @@ int hga_debug_timeline(unsigned long long* out, int max) {
   cudaMemcpyToSymbol(hga::g_tl_n, &zero, sizeof(zero));
   return (int)n;
 }
+int hga_debug_route_times(unsigned long long* out, int max) {
+  cudaDeviceSynchronize();
+  const int n = max < 4 * 4096 ? max : 4 * 4096;
+  cudaMemcpyFromSymbol(out, hga::g_rt, n * sizeof(unsigned long long));
+  return n;
+}
+int hga_debug_cta_times(unsigned long long* out, int max) {
+  cudaDeviceSynchronize();
+  const int n = max < 3 * 4096 ? max : 3 * 4096;
+  cudaMemcpyFromSymbol(out, hga::g_cta, n * sizeof(unsigned long long));
+  return n;
+}
 #endif
+
+hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return HGA_ERR_INVALID_ARG;
+  if (n == 0) return HGA_OK;
+  const int64_t pairs = (n + 1) / 2;
+  const unsigned blocks = (unsigned)std::min<int64_t>((pairs + 255) / 256, 1 << 20);
+  hga::exp2_selftest_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return after_launch();
+}
 
 hga_status hga_set_kernel_variant(int32_t variant) {
   if (variant < 0 || variant > 2) return HGA_ERR_INVALID_ARG;

@@ -375,6 +375,40 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
   }
 }
 
+// Kept chunks of (b, h) from the chunk router's output, compacted into smem:
+// entry i is kept when it lies in the candidate window [lo, hi) and exceeds
+// entry i-1 (the list must be strictly ascending).  Anything else is reported
+// (HGA_ERR_DEVICE_CHECK) and dropped.  All 256 threads load and test entries
+// in parallel; returns the count.
+__device__ int compact_kept_chunks(const RouteArgs& a, int b, int h, int lo, int64_t hi,
+                                   int* kept, int* s_n, int* tmp) {
+  const int32_t* in = a.in_idx + ((int64_t)h * a.n_blocks + b) * a.in_cap;
+  int cnt = a.in_cnt[(int64_t)h * a.n_blocks + b];
+  if (cnt < 0 || cnt > a.in_cap || cnt > 2048) {
+    if (threadIdx.x == 0) report(HGA_ERR_DEVICE_CHECK);
+    cnt = 0;
+  }
+  int base = 0;
+  for (int i0 = 0; i0 < cnt; i0 += kRouteThreads) {
+    const int i = i0 + threadIdx.x;
+    int c = -1;
+    bool ok = false;
+    if (i < cnt) {
+      c = in[i];
+      const int prev = i > 0 ? in[i - 1] : -1;
+      ok = c >= lo && c < hi && c > prev;
+      if (!ok) report(HGA_ERR_DEVICE_CHECK);
+    }
+    int total;
+    const int pos = block_excl_scan(ok ? 1 : 0, tmp, &total);
+    if (ok) kept[base + pos] = c;
+    base += total;
+  }
+  if (threadIdx.x == 0) *s_n = base;
+  __syncthreads();
+  return *s_n;
+}
+
 // ---------------------------------------------------------------- kernel
 
 template <typename T, int D>
@@ -398,23 +432,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   if (!a.group_mode) {
     cd.n = hi > cd.lo ? (int)(hi - cd.lo) : 0;
   } else {
-    // compact the valid kept chunks (ascending, inside the candidate window)
-    if (threadIdx.x == 0) {
-      const int32_t* in = a.in_idx + ((int64_t)h * a.n_blocks + b) * a.in_cap;
-      int cnt = a.in_cnt[(int64_t)h * a.n_blocks + b];
-      if (cnt < 0 || cnt > a.in_cap || cnt > 2048) { report(HGA_ERR_DEVICE_CHECK); cnt = 0; }
-      int m = 0, prev = -1;
-      for (int i = 0; i < cnt; ++i) {
-        const int c = in[i];
-        if (c < cd.lo || c >= hi || c <= prev) { report(HGA_ERR_DEVICE_CHECK); continue; }
-        s_kept[m++] = c;
-        prev = c;
-      }
-      s_nkept = m;
-    }
-    __syncthreads();
+    cd.n = compact_kept_chunks(a, b, h, cd.lo, hi, s_kept, &s_nkept, tmp) * cd.per;
     cd.kept = s_kept;
-    cd.n = s_nkept * cd.per;
   }
   const int k_eff = a.top_k <= 0 ? cd.n : min(a.top_k, cd.n);
   int32_t* out = a.out_idx + ((int64_t)h * a.n_blocks + b) * a.out_cap;

@@ -49,6 +49,12 @@ struct RtBars {
   int abort;
 };
 
+#ifdef HGA_TIMELINE
+// Debug builds only: per-CTA globaltimer stamps (start, scoring start,
+// scoring end, selection end).
+__device__ unsigned long long g_rt[4 * 4096];
+#endif
+
 struct RtArgs {
   RouteArgs r;
   int rs;            // query rows per slice (MMA N): min(256, 64 * G)
@@ -74,6 +80,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __shared__ int tmp[32];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+#ifdef HGA_TIMELINE
+  if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096)
+    g_rt[4 * (blockIdx.y * gridDim.x + blockIdx.x)] = tc::globaltimer_ns();
+#endif
   const int b = blockIdx.x, h = blockIdx.y;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
   const int npos = (int)min((int64_t)a.qblock, a.q_start + a.n_q - b0);
@@ -88,22 +98,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   if (!a.group_mode) {
     cd.n = hi > cd.lo ? (int)(hi - cd.lo) : 0;
   } else {
-    if (tid == 0) {
-      const int32_t* in = a.in_idx + ((int64_t)h * a.n_blocks + b) * a.in_cap;
-      int cnt = a.in_cnt[(int64_t)h * a.n_blocks + b];
-      if (cnt < 0 || cnt > a.in_cap || cnt > 2048) { report(HGA_ERR_DEVICE_CHECK); cnt = 0; }
-      int m = 0, prev = -1;
-      for (int i = 0; i < cnt; ++i) {
-        const int c = in[i];
-        if (c < cd.lo || c >= hi || c <= prev) { report(HGA_ERR_DEVICE_CHECK); continue; }
-        s_kept[m++] = c;
-        prev = c;
-      }
-      s_nkept = m;
-    }
-    __syncthreads();
+    cd.n = compact_kept_chunks(a, b, h, cd.lo, hi, s_kept, &s_nkept, tmp) * cd.per;
     cd.kept = s_kept;
-    cd.n = s_nkept * cd.per;
   }
   const int k_eff = a.top_k <= 0 ? cd.n : min(a.top_k, cd.n);
   int32_t* out = a.out_idx + ((int64_t)h * a.n_blocks + b) * a.out_cap;
@@ -120,6 +116,10 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
 
   // ---- scoring on the tensor cores
+#ifdef HGA_TIMELINE
+  if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096)
+    g_rt[4 * (blockIdx.y * gridDim.x + blockIdx.x) + 1] = tc::globaltimer_ns();
+#endif
   const int n_slices = (nrows + RS - 1) / RS;
   const int n_tiles = (cd.n + kRtTile - 1) / kRtTile;
   const int n_jobs = n_tiles * n_slices;
@@ -212,13 +212,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
           if (q >= 2 && !(ok = tc::mbar_wait(&bars->acc_empty[buf], ((q >> 1) - 1) & 1, abort_flag)))
             break;
           tc::fence_after_sync();
-          for (int k = 0; k < D / 16; ++k) {
-            const int hf = k >> 2, kk = k & 3;
-            const uint64_t ad = tc::sdesc_sw128(tc::smem_addr(stage(s, hf)) + kk * 32, 16, 1024);
-            const uint64_t bd = tc::sdesc_sw128(q_base + (r * L::kHalves + hf) * L::kQHalf + kk * 32,
-                                                16, 1024);
-            tc::mma_ss(tmem + buf * 256, ad, bd, idesc, k > 0);
-          }
+          // base descriptors once; k-steps move only the start address
+          const uint64_t ad0 = tc::sdesc_sw128(tc::smem_addr(stage(s, 0)), 16, 1024);
+          const uint64_t bd0 = tc::sdesc_sw128(q_base + r * L::kHalves * L::kQHalf, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k)
+            tc::mma_ss(tmem + buf * 256,
+                       ad0 + (uint64_t)((((k >> 2) * L::kTileHalf) + (k & 3) * 32) >> 4),
+                       bd0 + (uint64_t)((((k >> 2) * L::kQHalf) + (k & 3) * 32) >> 4), idesc, k > 0);
           tc::mma_commit(&bars->acc_full[buf]);
         }
         if (ok) tc::mma_commit(&bars->empty[s]);
@@ -239,18 +240,22 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       if (!tc::mbar_wait(&bars->acc_full[buf], (q >> 1) & 1, abort_flag)) break;
       tc::fence_after_sync();
       const int valid_cols = min(RS, nrows - r * RS);    // rows past the block: masked
+      // up to 128 columns in flight per TMEM round trip (RS is 64, 128 or 256)
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      for (int c0 = 0; c0 < RS; c0 += 32) {
-        uint32_t v[32];
-        tc::tmem_ld32(tmem + lane_off + buf * 256 + c0, v);
-        tc::tmem_wait_ld();
-        if (c0 + 32 <= valid_cols) {
+      for (int c0 = 0; c0 < RS; c0 += 128) {
+        uint32_t v[128];
+        const int nld = min(128, RS - c0) / 32;
 #pragma unroll
-          for (int x = 0; x < 32; ++x) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(v[x]));
+        for (int x = 0; x < 4; ++x)
+          if (x < nld) tc::tmem_ld32(tmem + lane_off + buf * 256 + c0 + 32 * x, v + 32 * x);
+        tc::tmem_wait_ld();
+        if (c0 + 128 <= valid_cols && nld == 4) {
+#pragma unroll
+          for (int x = 0; x < 128; ++x) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(v[x]));
         } else {
 #pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (c0 + x < valid_cols) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(v[x]));
+          for (int x = 0; x < 128; ++x)
+            if (x < 32 * nld && c0 + x < valid_cols) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(v[x]));
         }
       }
       tc::fence_before_sync();
@@ -270,7 +275,14 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     tc::tmem_dealloc(tmem, 512);
   }
   if (*abort_flag) return;
+#ifdef HGA_TIMELINE
+  const int cta_l = blockIdx.y * gridDim.x + blockIdx.x;
+  if (tid == 0 && cta_l < 4096) g_rt[4 * cta_l + 2] = tc::globaltimer_ns();
+#endif
   select_emit(sc, cd, k_eff, out, hist, tmp);
+#ifdef HGA_TIMELINE
+  if (tid == 0 && cta_l < 4096) g_rt[4 * cta_l + 3] = tc::globaltimer_ns();
+#endif
 }
 
 }  // namespace hga

@@ -217,6 +217,60 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------- packed f32x2
+
+// Two floats in one 64-bit register pair (sm_100 packed FP32 arithmetic:
+// one instruction does two lanes' worth of FMA / ADD).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair of floats on the FMA pipe (to share the load of the MUFU
+// unit).  Cody-Waite reduction (W. J. Cody and W. Waite, "Software Manual for
+// the Elementary Functions", 1980): j = round(x) by adding 1.5 * 2^23, f =
+// x - j in [-1/2, 1/2]; 2^f by a degree-4 polynomial (near-minimax least
+// squares on Chebyshev nodes, fitted by csrc/exp2_poly.py, max relative error
+// 2.7e-6 in float32); 2^j added to the exponent field.  x is clamped to
+// >= -125 first (-inf gives 2^-125, which rounds to 0 in fp16).  Valid for
+// x <= 127.
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
+  float x0, x1;
+  unpk2(x, x0, x1);
+  x = pk2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = pk2(12582912.f, 12582912.f);      // 1.5 * 2^23
+  const uint64_t t = fadd2(x, magic);                       // j in the low bits
+  const uint64_t jj = fadd2(t, pk2(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(jj, pk2(-1.f, -1.f), x);          // x - j
+  uint64_t p = pk2(0.00956051052f, 0.00956051052f);
+  p = ffma2(p, f, pk2(0.0559170395f, 0.0559170395f));
+  p = ffma2(p, f, pk2(0.240249813f, 0.240249813f));
+  p = ffma2(p, f, pk2(0.69312197f, 0.69312197f));
+  p = ffma2(p, f, pk2(0.999999166f, 0.999999166f));
+  float p0, p1, t0, t1;
+  unpk2(p, p0, p1);
+  unpk2(t, t0, t1);
+  // exponent field += j: the low 32 bits of t hold 0x4B400000 + j, so
+  // (bits(t) << 23) == j << 23 modulo 2^32
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return pk2(r0, r1);
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;\n" : "=r"(r) : "f"(b), "f"(a));
@@ -224,4 +278,18 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 }  // namespace tc
+
+// y[i] = tc::exp2_fma2(x[i]) (pairs; a trailing odd element pairs with 0).
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                     int64_t n) {
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; 2 * p < n;
+       p += (int64_t)gridDim.x * blockDim.x) {
+    const float a = x[2 * p], b = 2 * p + 1 < n ? x[2 * p + 1] : 0.f;
+    float r0, r1;
+    tc::unpk2(tc::exp2_fma2(tc::pk2(a, b)), r0, r1);
+    y[2 * p] = r0;
+    if (2 * p + 1 < n) y[2 * p + 1] = r1;
+  }
+}
+
 }  // namespace hga

@@ -25,7 +25,7 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_attend", "hga_forward", "hga_index_capacity",
             "hga_validate_params", "hga_check", "hga_status_string",
             "hga_launch_count", "hga_last_cuda_error",
-            "hga_set_kernel_variant")
+            "hga_set_kernel_variant", "hga_selftest_exp2")
 
 
 class HgaError(RuntimeError):
@@ -94,6 +94,7 @@ def _load() -> ctypes.CDLL:
         "hga_launch_count": [],
         "hga_last_cuda_error": [],
         "hga_set_kernel_variant": [i32],
+        "hga_selftest_exp2": [vp, vp, i64, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -230,3 +231,11 @@ def allocate(p: Params, t_cap: int, n_q: int, device="cuda",
 def set_kernel_variant(variant: int):
     """0 = automatic (tcgen05 kernel when eligible), 1 = portable mma.sync."""
     _ok(LIB.hga_set_kernel_variant(variant), "hga_set_kernel_variant")
+
+
+def selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The attention kernel's software 2^x applied to a float32 device tensor."""
+    y = torch.empty_like(x)
+    _ok(LIB.hga_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+        "hga_selftest_exp2")
+    return y

@@ -20,7 +20,7 @@ def hga():
 def _declared():
     src = open(os.path.join(ROOT, "include", "hga.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(hga_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b(hga_[a-z_0-9]+)\s*\(", src)))
 
 
 def test_exports_every_declared_symbol(hga):

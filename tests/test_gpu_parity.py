@@ -155,3 +155,19 @@ def test_attend_variants_agree_with_oracle(variant):
         _check(gi.QWEN3_30B_64K.with_(T=4136, q0=2048, n_needles=8))
     finally:
         hga.set_kernel_variant(0)
+
+
+def test_software_exp2_matches_cuda_exp2f():
+    """The FMA-pipe 2^x used for part of each softmax row stays within 3e-6
+    relative of CUDA's exp2f over the range the kernel feeds it, and gives
+    ~0 for -inf (masked scores)."""
+    from long_context_hga_b200 import hga
+    x = torch.linspace(-125.0, 8.0, 1 << 20, device="cuda", dtype=torch.float32)
+    x = torch.cat([x, torch.rand(1 << 18, device="cuda") * 16 - 8,
+                   torch.tensor([0.0, -0.5, 0.5, 7.99, -124.9], device="cuda")])
+    y = hga.selftest_exp2(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel < 3e-6, rel
+    z = hga.selftest_exp2(torch.tensor([-float("inf"), -1e30, -200.0], device="cuda"))
+    assert (z >= 0).all() and (z < 3e-38).all()
