@@ -156,6 +156,54 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start,
                        int32_t* group_idx, int32_t* group_cnt, void* o,
                        float* lse, hga_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Host-memory tier ("Long-Context Fine-Tuning with Limited VRAM", section 2.2
+ * tiered KV storage; section 2.1 group summaries in a VRAM cache with misses
+ * fetched from RAM; section 4.5 cache hit rate).  History = tokens < t_hist
+ * (a multiple of group, <= q_start).  Its K/V and all group summaries live in
+ * pinned host memory (readable by the device: page-locked, unified
+ * addressing), [n_kv_heads][t_cap][head_dim] and [n_kv_heads][t_cap/group]
+ * [head_dim].  Device "mirrors" with the all-HBM layouts receive what a step
+ * needs, so hga_route_groups and hga_attend run on them unchanged:
+ *   route chunks -> hga_fetch_group_summaries -> hga_route_groups
+ *   -> hga_gather_history (may run on a side stream; hga_attend waits)
+ *   -> hga_attend -> hga_install_group_cache.
+ * Results equal the all-HBM path's exactly. */
+typedef struct hga_group_cache {
+  void* data;                  /* device [n_kv_heads][cap][head_dim], dtype       */
+  int32_t* tags;               /* device [n_kv_heads][cap]: group held, -1 empty  */
+  int32_t* claims;             /* device [n_kv_heads][cap]: largest group that    */
+                               /*   missed on the slot this step, -1 none         */
+  int64_t cap;                 /* slots per KV head; group j maps to j % cap      */
+  unsigned long long* stats;   /* device [2] hits, misses (accumulated), nullable */
+} hga_group_cache;
+
+/* Group summaries of every kept history chunk of every (block, KV head) are
+ * copied into group_sum_dev: from the cache on a hit, from group_sum_host on
+ * a miss (the slot is then claimed).  tags/claims start at -1 (caller). */
+hga_status hga_fetch_group_summaries(const hga_params* p, int64_t q_start, int64_t n_q,
+                                     int64_t t_cap, int64_t t_hist, const int32_t* chunk_idx,
+                                     const int32_t* chunk_cnt, const void* group_sum_host,
+                                     const hga_group_cache* cache, void* group_sum_dev,
+                                     hga_stream_t stream);
+
+/* Copies the history K/V groups the step attends (sink, routed, local window,
+ * below t_hist) from k_host/v_host into k_dev/v_dev, each (KV head, group) at
+ * most once per step: gen ([n_kv_heads][t_cap/group] uint32, zero at first
+ * use) is stamped with `step` (nonzero, distinct per call).  Adds the bytes
+ * copied to *bytes when bytes != NULL. */
+hga_status hga_gather_history(const hga_params* p, int64_t q_start, int64_t n_q, int64_t t_cap,
+                              int64_t t_hist, const int32_t* group_idx, const int32_t* group_cnt,
+                              const void* k_host, const void* v_host, void* k_dev, void* v_dev,
+                              uint32_t* gen, uint32_t step, unsigned long long* bytes,
+                              hga_stream_t stream);
+
+/* Every claimed cache slot takes its claim (summary copied from
+ * group_sum_host, tag set, claim cleared).  Run after the step's lookups. */
+hga_status hga_install_group_cache(const hga_params* p, int64_t t_cap,
+                                   const void* group_sum_host, const hga_group_cache* cache,
+                                   hga_stream_t stream);
+
 /* Slots per (KV head, block) of chunk_idx (which = 0) or group_idx
  * (which = 1) for a context capacity t_cap; -1 on invalid parameters. */
 int64_t hga_index_capacity(const hga_params* p, int64_t t_cap, int32_t which);

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
   int* list = reinterpret_cast<int*>(sv + 2 * kAttTok * D * 2);
   __shared__ bool s_invalid;
 
+  griddep_wait();
   const int tile_r = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
@@ -324,6 +325,7 @@ __global__ void __launch_bounds__(256) attend_f32_kernel(AttendArgs a) {
   extern __shared__ __align__(128) char smem[];
   int* list = reinterpret_cast<int*>(smem);
   __shared__ bool s_invalid;
+  griddep_wait();
   const int tile_r = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;

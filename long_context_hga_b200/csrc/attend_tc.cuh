@@ -111,6 +111,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* list = reinterpret_cast<int*>(smem + L::kListOff);
   volatile int* abort_flag = &bars->abort;
 
+  griddep_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.y, h = blockIdx.z;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
@@ -542,6 +543,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // ---- teardown: all roles done (every wait above is bounded)
+  griddep_launch();
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {

@@ -15,6 +15,19 @@ __device__ int g_status;
 
 __device__ __forceinline__ void report(int code) { atomicCAS(&g_status, 0, code); }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while the previous kernel of the stream is finishing;
+// griddep_wait() blocks until that kernel has completed and its writes are
+// visible (call it before reading any input), griddep_launch() lets the next
+// kernel start launching (called once a CTA's main work is done).  Both are
+// no-ops without the launch attribute.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // ---------------------------------------------------------------- rounding
 
 // float64 -> bfloat16, round to nearest even, in one rounding: round to odd

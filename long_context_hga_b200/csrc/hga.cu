@@ -15,6 +15,7 @@
 #include "attend.cuh"
 #include "attend_tc.cuh"
 #include "route_tc.cuh"
+#include "tier.cuh"
 
 namespace {
 
@@ -29,6 +30,31 @@ inline hga_status cuda_ok(cudaError_t e) {
 
 inline hga_status after_launch() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cuda_ok(cudaGetLastError());
+}
+
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel on the stream drains; the kernels call
+// griddepcontrol.wait before reading anything (see common.cuh).
+template <typename... KArgs, typename... Args>
+hga_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_ok(e);
+  }
   return cuda_ok(cudaGetLastError());
 }
 
@@ -147,8 +173,8 @@ hga_status launch_route_tc(hga::RouteArgs& a, cudaStream_t st) {
       !encode_bf16_map(&ts8, a.summ, 2, sd, ss, sb8))
     return HGA_ERR_CUDA;
   dim3 grid(a.n_blocks, a.Hkv);
-  hga::route_tc_kernel<D><<<grid, hga::kRtThreads, L::kSmem, st>>>(tq, ts, ts8, ra);
-  return after_launch();
+  return launch_pdl(hga::route_tc_kernel<D>, grid, dim3(hga::kRtThreads), L::kSmem, st, tq, ts,
+                    ts8, ra);
 }
 
 constexpr int kMaxRouteCands = 16384;
@@ -160,8 +186,7 @@ hga_status launch_route(hga::RouteArgs& a, cudaStream_t st) {
   hga_status s = allow_smem<hga::route_kernel<T, D>>(smem);
   if (s != HGA_OK) return s;
   dim3 grid(a.n_blocks, a.Hkv);
-  hga::route_kernel<T, D><<<grid, hga::kRouteThreads, smem, st>>>(a);
-  return after_launch();
+  return launch_pdl(hga::route_kernel<T, D>, grid, dim3(hga::kRouteThreads), smem, st, a);
 }
 
 hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
@@ -232,10 +257,9 @@ hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_beg
   (void)chunk;
   (void)group;   // 64 / 8, validated by check_params
   dim3 grid((unsigned)n_chunks, Hkv);
-  hga::summaries_kernel<T, D><<<grid, 32 * hga::kSumGroupsPerChunk, 0, st>>>(
-      reinterpret_cast<const T*>(k), t_cap, c_first, t_end, reinterpret_cast<T*>(cs),
-      reinterpret_cast<T*>(gs));
-  return after_launch();
+  return launch_pdl(hga::summaries_kernel<T, D>, grid, dim3(32 * hga::kSumGroupsPerChunk), 0, st,
+                    reinterpret_cast<const T*>(k), t_cap, c_first, t_end, reinterpret_cast<T*>(cs),
+                    reinterpret_cast<T*>(gs));
 }
 
 template <int D>
@@ -260,8 +284,8 @@ hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
     return HGA_ERR_CUDA;
   hga::TcArgs ta{a, 2 * hga::kTcRows};
   dim3 grid((a.qblock * a.G + ta.rows_per_cta - 1) / ta.rows_per_cta, a.n_blocks, a.Hkv);
-  hga::attend_tc_kernel<D><<<grid, hga::kTcThreads, smem, st>>>(tq, tk1, tk8, tv1, tv8, ta);
-  return after_launch();
+  return launch_pdl(hga::attend_tc_kernel<D>, grid, dim3(hga::kTcThreads), smem, st, tq, tk1, tk8,
+                    tv1, tv8, ta);
 }
 
 bool tc_eligible(const hga::AttendArgs& a) {
@@ -280,8 +304,7 @@ hga_status launch_attend_bf16(hga::AttendArgs& a, cudaStream_t st) {
   hga_status s = allow_smem<hga::attend_mma_kernel<D>>(smem);
   if (s != HGA_OK) return s;
   dim3 grid((a.qblock * a.G + hga::kAttRows - 1) / hga::kAttRows, a.n_blocks, a.Hkv);
-  hga::attend_mma_kernel<D><<<grid, 128, smem, st>>>(a);
-  return after_launch();
+  return launch_pdl(hga::attend_mma_kernel<D>, grid, dim3(128), smem, st, a);
 }
 
 template <int D>
@@ -290,8 +313,7 @@ hga_status launch_attend_f32(hga::AttendArgs& a, cudaStream_t st) {
   hga_status s = allow_smem<hga::attend_f32_kernel<D>>(smem);
   if (s != HGA_OK) return s;
   dim3 grid((a.qblock * a.G + hga::kAttF32Rows - 1) / hga::kAttF32Rows, a.n_blocks, a.Hkv);
-  hga::attend_f32_kernel<D><<<grid, 256, smem, st>>>(a);
-  return after_launch();
+  return launch_pdl(hga::attend_f32_kernel<D>, grid, dim3(256), smem, st, a);
 }
 
 }  // namespace
@@ -451,6 +473,120 @@ int hga_debug_cta_times(unsigned long long* out, int max) {
   return n;
 }
 #endif
+
+// ---------------------------------------------------------------- host tier
+
+static hga_status tier_args(const hga_params* p, int64_t q_start, int64_t n_q, int64_t t_cap,
+                            int64_t t_hist, hga::TierArgs* a) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
+  if (t_hist < 0 || t_hist > q_start || t_hist % p->group) return HGA_ERR_INVALID_ARG;
+  *a = hga::TierArgs{};
+  a->q_start = q_start;
+  a->n_q = n_q;
+  a->t_cap = t_cap;
+  a->t_hist = t_hist;
+  a->n_blocks = (int)((n_q + p->qblock - 1) / p->qblock);
+  a->Hkv = p->n_kv_heads;
+  a->chunk = p->chunk;
+  a->group = p->group;
+  a->qblock = p->qblock;
+  a->sink = p->sink;
+  a->local = p->local;
+  a->n_groups_cap = t_cap / p->group;
+  a->in_cap = cap_chunks(p, t_cap);
+  a->cap_g = cap_groups(p, t_cap);
+  return HGA_OK;
+}
+
+hga_status hga_fetch_group_summaries(const hga_params* p, int64_t q_start, int64_t n_q,
+                                     int64_t t_cap, int64_t t_hist, const int32_t* chunk_idx,
+                                     const int32_t* chunk_cnt, const void* group_sum_host,
+                                     const hga_group_cache* cache, void* group_sum_dev,
+                                     hga_stream_t stream) {
+  hga::TierArgs a;
+  hga_status s = tier_args(p, q_start, n_q, t_cap, t_hist, &a);
+  if (s != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!chunk_idx || !chunk_cnt || !group_sum_host || !cache || !group_sum_dev || !cache->data ||
+      !cache->tags || !cache->claims || cache->cap <= 0 || cache->cap > 0x7fffffff)
+    return HGA_ERR_INVALID_ARG;
+  a.cache_cap = cache->cap;
+  dim3 grid(a.n_blocks, a.Hkv);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto go = [&](auto tag, auto dim) {
+    using T = decltype(tag);
+    constexpr int D = decltype(dim)::value;
+    return launch_pdl(hga::fetch_group_summaries_kernel<D, T>, grid, dim3(256), 0, st, a,
+                      chunk_idx, chunk_cnt, reinterpret_cast<const T*>(group_sum_host),
+                      reinterpret_cast<const T*>(cache->data), (const int32_t*)cache->tags,
+                      cache->claims, reinterpret_cast<T*>(group_sum_dev), cache->stats);
+  };
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? go(__nv_bfloat16{}, std::integral_constant<int, 128>{})
+                              : go(__nv_bfloat16{}, std::integral_constant<int, 64>{});
+  return p->head_dim == 128 ? go(float{}, std::integral_constant<int, 128>{})
+                            : go(float{}, std::integral_constant<int, 64>{});
+}
+
+hga_status hga_gather_history(const hga_params* p, int64_t q_start, int64_t n_q, int64_t t_cap,
+                              int64_t t_hist, const int32_t* group_idx, const int32_t* group_cnt,
+                              const void* k_host, const void* v_host, void* k_dev, void* v_dev,
+                              uint32_t* gen, uint32_t step, unsigned long long* bytes,
+                              hga_stream_t stream) {
+  hga::TierArgs a;
+  hga_status s = tier_args(p, q_start, n_q, t_cap, t_hist, &a);
+  if (s != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!group_idx || !group_cnt || !k_host || !v_host || !k_dev || !v_dev || !gen || step == 0)
+    return HGA_ERR_INVALID_ARG;
+  dim3 grid(a.n_blocks, a.Hkv);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto go = [&](auto tag, auto dim) {
+    using T = decltype(tag);
+    constexpr int D = decltype(dim)::value;
+    return launch_pdl(hga::gather_history_kernel<D, T>, grid, dim3(256), 0, st, a, group_idx,
+                      group_cnt, reinterpret_cast<const T*>(k_host),
+                      reinterpret_cast<const T*>(v_host), reinterpret_cast<T*>(k_dev),
+                      reinterpret_cast<T*>(v_dev), gen, step, bytes);
+  };
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? go(__nv_bfloat16{}, std::integral_constant<int, 128>{})
+                              : go(__nv_bfloat16{}, std::integral_constant<int, 64>{});
+  return p->head_dim == 128 ? go(float{}, std::integral_constant<int, 128>{})
+                            : go(float{}, std::integral_constant<int, 64>{});
+}
+
+hga_status hga_install_group_cache(const hga_params* p, int64_t t_cap,
+                                   const void* group_sum_host, const hga_group_cache* cache,
+                                   hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if (t_cap <= 0 || !group_sum_host || !cache || !cache->data || !cache->tags || !cache->claims ||
+      cache->cap <= 0 || cache->cap > 0x7fffffff)
+    return HGA_ERR_INVALID_ARG;
+  hga::TierArgs a{};
+  a.Hkv = p->n_kv_heads;
+  a.n_groups_cap = t_cap / p->group;
+  a.cache_cap = cache->cap;
+  const int64_t warps = (int64_t)a.Hkv * a.cache_cap;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks > 0x7fffffff) return HGA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto go = [&](auto tag, auto dim) {
+    using T = decltype(tag);
+    constexpr int D = decltype(dim)::value;
+    return launch_pdl(hga::install_group_cache_kernel<D, T>, dim3((unsigned)blocks), dim3(256), 0,
+                      st, a, reinterpret_cast<const T*>(group_sum_host),
+                      reinterpret_cast<T*>(cache->data), cache->tags, cache->claims);
+  };
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? go(__nv_bfloat16{}, std::integral_constant<int, 128>{})
+                              : go(__nv_bfloat16{}, std::integral_constant<int, 64>{});
+  return p->head_dim == 128 ? go(float{}, std::integral_constant<int, 128>{})
+                            : go(float{}, std::integral_constant<int, 64>{});
+}
 
 hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t stream) {
   if (n < 0 || (n > 0 && (!x || !y))) return HGA_ERR_INVALID_ARG;

@@ -414,6 +414,7 @@ __device__ int compact_kept_chunks(const RouteArgs& a, int b, int h, int lo, int
 template <typename T, int D>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   extern __shared__ __align__(128) char smem[];
+  griddep_wait();
   const int b = blockIdx.x, h = blockIdx.y;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
   const int npos = (int)min((int64_t)a.qblock, a.q_start + a.n_q - b0);
@@ -461,6 +462,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
       score_f32<D>(a, b, h, (int)b0, nrows, cd, sc, sq, stile, red);
     }
   }
+  griddep_launch();
   select_emit(sc, cd, k_eff, out, hist, tmp);
 }
 

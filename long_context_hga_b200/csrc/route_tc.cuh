@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096)
     g_rt[4 * (blockIdx.y * gridDim.x + blockIdx.x)] = tc::globaltimer_ns();
 #endif
+  griddep_wait();
   const int b = blockIdx.x, h = blockIdx.y;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
   const int npos = (int)min((int64_t)a.qblock, a.q_start + a.n_q - b0);
@@ -275,6 +276,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     tc::tmem_dealloc(tmem, 512);
   }
   if (*abort_flag) return;
+  griddep_launch();
 #ifdef HGA_TIMELINE
   const int cta_l = blockIdx.y * gridDim.x + blockIdx.x;
   if (tid == 0 && cta_l < 4096) g_rt[4 * cta_l + 2] = tc::globaltimer_ns();

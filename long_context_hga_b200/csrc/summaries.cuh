@@ -32,6 +32,8 @@ __global__ void __launch_bounds__(32 * kSumGroupsPerChunk) summaries_kernel(
   constexpr int kChunk = kSumGroup * kSumGroupsPerChunk;
   __shared__ double s_gsum[kSumGroupsPerChunk][D];
 
+  griddep_wait();
+  griddep_launch();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.y;
   const int64_t c = c_first + blockIdx.x;

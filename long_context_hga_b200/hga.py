@@ -25,7 +25,8 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_attend", "hga_forward", "hga_index_capacity",
             "hga_validate_params", "hga_check", "hga_status_string",
             "hga_launch_count", "hga_last_cuda_error",
-            "hga_set_kernel_variant", "hga_selftest_exp2")
+            "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
+            "hga_gather_history", "hga_install_group_cache")
 
 
 class HgaError(RuntimeError):
@@ -239,3 +240,118 @@ def selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
     _ok(LIB.hga_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
         "hga_selftest_exp2")
     return y
+
+
+# ---------------------------------------------------------------- host tier
+
+class CGroupCache(ctypes.Structure):
+    _fields_ = [("data", ctypes.c_void_p), ("tags", ctypes.c_void_p),
+                ("claims", ctypes.c_void_p), ("cap", ctypes.c_int64),
+                ("stats", ctypes.c_void_p)]
+
+
+def _sig_tier():
+    P = ctypes.POINTER(CParams)
+    vp, i64, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint32
+    C = ctypes.POINTER(CGroupCache)
+    LIB.hga_fetch_group_summaries.argtypes = [P, i64, i64, i64, i64, vp, vp, vp, C, vp, vp]
+    LIB.hga_gather_history.argtypes = [P, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, u32,
+                                       vp, vp]
+    LIB.hga_install_group_cache.argtypes = [P, i64, vp, C, vp]
+    for n in ("hga_fetch_group_summaries", "hga_gather_history", "hga_install_group_cache"):
+        getattr(LIB, n).restype = ctypes.c_int
+
+
+_sig_tier()
+
+
+@dataclasses.dataclass
+class HostTier:
+    """History K/V and group summaries in pinned host memory, an HBM cache of
+    group summaries (direct mapped), and device mirrors that routing and
+    attention read."""
+    t_hist: int
+    k_host: torch.Tensor
+    v_host: torch.Tensor
+    gsum_host: torch.Tensor
+    cache_data: torch.Tensor
+    tags: torch.Tensor
+    claims: torch.Tensor
+    stats: torch.Tensor          # int64 [2]: hits, misses
+    gen: torch.Tensor            # int32 [Hkv][t_cap/group] generation stamps
+    bytes: torch.Tensor          # int64 [1]: history bytes gathered
+    step: int = 0
+
+    def c_cache(self) -> CGroupCache:
+        return CGroupCache(self.cache_data.data_ptr(), self.tags.data_ptr(),
+                           self.claims.data_ptr(), self.tags.shape[1],
+                           self.stats.data_ptr())
+
+
+def make_host_tier(p: Params, k_host: torch.Tensor, v_host: torch.Tensor,
+                   gsum_host: torch.Tensor, t_hist: int, cache_fraction: float = 0.25,
+                   device="cuda") -> HostTier:
+    """k_host/v_host/gsum_host: pinned CPU tensors in the all-HBM layouts."""
+    for t in (k_host, v_host, gsum_host):
+        if not t.is_pinned():
+            raise ValueError("host tier tensors must be pinned")
+    Hkv, n_groups = gsum_host.shape[0], gsum_host.shape[1]
+    cap = max(1, int(-(-cache_fraction * Hkv * n_groups // Hkv)))
+    return HostTier(
+        t_hist=t_hist, k_host=k_host, v_host=v_host, gsum_host=gsum_host,
+        cache_data=torch.zeros(Hkv, cap, p.head_dim, dtype=p.torch_dtype, device=device),
+        tags=torch.full((Hkv, cap), -1, dtype=torch.int32, device=device),
+        claims=torch.full((Hkv, cap), -1, dtype=torch.int32, device=device),
+        stats=torch.zeros(2, dtype=torch.int64, device=device),
+        gen=torch.zeros(Hkv, n_groups, dtype=torch.int32, device=device),
+        bytes=torch.zeros(1, dtype=torch.int64, device=device))
+
+
+def fetch_group_summaries(p: Params, q_start: int, n_q: int, t_cap: int,
+                          tier: HostTier, chunk_idx, chunk_cnt, group_sum_dev,
+                          stream=None):
+    c = tier.c_cache()
+    _ok(LIB.hga_fetch_group_summaries(
+        ctypes.byref(p.c()), q_start, n_q, t_cap, tier.t_hist, _ptr(chunk_idx),
+        _ptr(chunk_cnt), _ptr(tier.gsum_host), ctypes.byref(c), _ptr(group_sum_dev),
+        _stream(stream)), "hga_fetch_group_summaries")
+
+
+def gather_history(p: Params, q_start: int, n_q: int, t_cap: int, tier: HostTier,
+                   group_idx, group_cnt, k_dev, v_dev, stream=None):
+    tier.step += 1
+    _ok(LIB.hga_gather_history(
+        ctypes.byref(p.c()), q_start, n_q, t_cap, tier.t_hist, _ptr(group_idx),
+        _ptr(group_cnt), _ptr(tier.k_host), _ptr(tier.v_host), _ptr(k_dev), _ptr(v_dev),
+        _ptr(tier.gen), ctypes.c_uint32(tier.step), _ptr(tier.bytes), _stream(stream)),
+        "hga_gather_history")
+
+
+def install_group_cache(p: Params, t_cap: int, tier: HostTier, stream=None):
+    c = tier.c_cache()
+    _ok(LIB.hga_install_group_cache(ctypes.byref(p.c()), t_cap, _ptr(tier.gsum_host),
+                                    ctypes.byref(c), _stream(stream)),
+        "hga_install_group_cache")
+
+
+def tiered_step(p: Params, q, q_start: int, tier: HostTier, k_dev, v_dev, bufs: "Buffers",
+                side_stream=None):
+    """One query segment through the tier: segment summaries, chunk routing,
+    summary fetch (cache / host), group routing, history gather on a side
+    stream, attention, cache install.  k_dev/v_dev hold the segment's own K/V
+    at [q_start, q_start + n_q); bufs.group_sum is the device summary mirror."""
+    main = torch.cuda.current_stream()
+    side = side_stream or torch.cuda.Stream()
+    n_q, t_cap = q.shape[0], k_dev.shape[1]
+    build_summaries(p, k_dev, q_start, q_start + n_q, bufs.chunk_sum, bufs.group_sum)
+    route_chunks(p, q, q_start, bufs.chunk_sum, t_cap, bufs.chunk_idx, bufs.chunk_cnt)
+    fetch_group_summaries(p, q_start, n_q, t_cap, tier, bufs.chunk_idx, bufs.chunk_cnt,
+                          bufs.group_sum)
+    route_groups(p, q, q_start, bufs.group_sum, t_cap, bufs.chunk_idx, bufs.chunk_cnt,
+                 bufs.group_idx, bufs.group_cnt)
+    side.wait_stream(main)
+    gather_history(p, q_start, n_q, t_cap, tier, bufs.group_idx, bufs.group_cnt, k_dev,
+                   v_dev, stream=side)
+    main.wait_stream(side)
+    attend(p, q, q_start, k_dev, v_dev, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
+    install_group_cache(p, t_cap, tier)
