@@ -47,6 +47,35 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+ATTEND_SOURCES = ("attend_tc.cuh", "tc.cuh", "common.cuh")
+
+
+def profiled_traffic(workload: str, kernel: str = "attend_tc", sources=ATTEND_SOURCES):
+    """DRAM bytes per launch from the committed ncu summary of `kernel` on
+    `workload`, or None when there is none or the kernel's sources changed
+    since the counters were taken (the summary records their sha256)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith(" "):
+                key, _, val = line.partition(":")
+                fields[key.strip()] = val.strip()
+    h = hashlib.sha256()
+    for name in sources:
+        with open(os.path.join(ROOT, "long_context_hga_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    if fields.get("kernel_sources_sha256") != h.hexdigest():
+        return None
+    try:
+        return int(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 # ---------------------------------------------------------------- dist
 
 def dist_setup():
@@ -380,7 +409,8 @@ def run_hga(args, world, rank, local):
             "density": counts["density"],
             "roofline": {"bound": "tensor", "kernel": "hga_attend",
                          "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
-                         "frac": att_tflops / peak_tf, "traffic": None,
+                         "frac": att_tflops / peak_tf,
+                         "traffic": profiled_traffic(w.name),
                          "peak_source": f"{peak_kind} bf16 burst",
                          "algorithmic_flops": counts["attn_flops"],
                          "algorithmic_bytes": counts["attn_bytes"],
