@@ -204,6 +204,33 @@ hga_status hga_install_group_cache(const hga_params* p, int64_t t_cap,
                                    const void* group_sum_host, const hga_group_cache* cache,
                                    hga_stream_t stream);
 
+/* hga_gather_history without the caller's generation array.  The pages have
+ * no counterpart: this call exists for callers that cannot allocate device
+ * memory for the stamps, e.g. a runtime that sizes all device memory once at
+ * start-up, or a host with no CUDA allocator of its own.
+ * - Result: the same copies, in the same places, as one hga_gather_history
+ *   call with a zeroed gen array; *bytes (when not NULL) grows by the same
+ *   amount.
+ * - Storage: the stamps live in a fixed 1 MiB array in the library's device
+ *   memory. n_kv_heads * (t_cap / group) must be at most 262144, otherwise
+ *   HGA_ERR_UNSUPPORTED is returned before any launch. Every call first zeroes
+ *   the part it uses, so no state carries over between calls.
+ * - Allocation: none. No cudaMalloc or cudaFree, and no allocating library
+ *   call.
+ * - First call on a device: it looks up the array's device address once, with
+ *   that device current. That call must not be made while `stream` is being
+ *   captured; if it is, the call returns HGA_ERR_UNSUPPORTED and launches
+ *   nothing. Make the first call outside any capture.
+ * - Concurrency: one array per device. Calls whose executions overlap on one
+ *   device (other streams, other host threads) race on it and may skip or
+ *   repeat copies. Order them on one stream, or with events.
+ * - Other arguments and errors: as hga_gather_history. */
+hga_status hga_gather_history_noalloc(const hga_params* p, int64_t q_start, int64_t n_q,
+                                      int64_t t_cap, int64_t t_hist, const int32_t* group_idx,
+                                      const int32_t* group_cnt, const void* k_host,
+                                      const void* v_host, void* k_dev, void* v_dev,
+                                      unsigned long long* bytes, hga_stream_t stream);
+
 /* Slots per (KV head, block) of chunk_idx (which = 0) or group_idx
  * (which = 1) for a context capacity t_cap; -1 on invalid parameters. */
 int64_t hga_index_capacity(const hga_params* p, int64_t t_cap, int32_t which);

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdio>
+#include <mutex>
 
 #include "hga.h"
 #include "common.cuh"
@@ -16,6 +17,7 @@
 #include "attend_tc.cuh"
 #include "route_tc.cuh"
 #include "tier.cuh"
+#include "noalloc.cuh"
 
 namespace {
 
@@ -604,5 +606,67 @@ hga_status hga_set_kernel_variant(int32_t variant) {
 }
 
 const char* hga_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the history gather (see noalloc.cuh for which
+// callers need it).  The stamps live in hga::g_static_gen; its device address
+// is looked up once per device, with that device current, the first time the
+// call runs there.
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_gen_mu;
+uint32_t* g_static_gen_ptr[kMaxDevices] = {};
+
+hga_status static_gen_address(cudaStream_t st, uint32_t** out) {
+  int dev = -1;
+  hga_status s = cuda_ok(cudaGetDevice(&dev));
+  if (s != HGA_OK) return s;
+  if (dev < 0 || dev >= kMaxDevices) return HGA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_gen_mu);
+  if (!g_static_gen_ptr[dev]) {
+    // The lookup may load the module; it is not done while `st` is being
+    // captured into a graph.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if ((s = cuda_ok(cudaStreamIsCapturing(st, &cs))) != HGA_OK) return s;
+    if (cs != cudaStreamCaptureStatusNone) return HGA_ERR_UNSUPPORTED;
+    void* ptr = nullptr;
+    if ((s = cuda_ok(cudaGetSymbolAddress(&ptr, hga::g_static_gen))) != HGA_OK) return s;
+    g_static_gen_ptr[dev] = static_cast<uint32_t*>(ptr);
+  }
+  *out = g_static_gen_ptr[dev];
+  return HGA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+hga_status hga_gather_history_noalloc(const hga_params* p, int64_t q_start, int64_t n_q,
+                                      int64_t t_cap, int64_t t_hist, const int32_t* group_idx,
+                                      const int32_t* group_cnt, const void* k_host,
+                                      const void* v_host, void* k_dev, void* v_dev,
+                                      unsigned long long* bytes, hga_stream_t stream) {
+  hga::TierArgs a;
+  hga_status s = tier_args(p, q_start, n_q, t_cap, t_hist, &a);
+  if (s != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!group_idx || !group_cnt || !k_host || !v_host || !k_dev || !v_dev)
+    return HGA_ERR_INVALID_ARG;
+  const int64_t words = (int64_t)a.Hkv * a.n_groups_cap;
+  if (words > hga::kStaticGenWords) return HGA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* gen = nullptr;
+  if ((s = static_gen_address(st, &gen)) != HGA_OK) return s;
+  // Stamps left by an earlier call would read as "already copied": clear the
+  // range this call uses, then gather with stamp 1.
+  const unsigned blocks = (unsigned)std::min<int64_t>((words + 255) / 256, 148 * 8);
+  hga::clear_stamps_kernel<<<blocks, 256, 0, st>>>(gen, words);
+  if ((s = after_launch()) != HGA_OK) return s;
+  return hga_gather_history(p, q_start, n_q, t_cap, t_hist, group_idx, group_cnt, k_host,
+                            v_host, k_dev, v_dev, gen, 1u, bytes, stream);
+}
 
 }  // extern "C"

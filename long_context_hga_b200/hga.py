@@ -26,7 +26,8 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_validate_params", "hga_check", "hga_status_string",
             "hga_launch_count", "hga_last_cuda_error",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
-            "hga_gather_history", "hga_install_group_cache")
+            "hga_gather_history", "hga_install_group_cache",
+            "hga_gather_history_noalloc")
 
 
 class HgaError(RuntimeError):
@@ -258,7 +259,10 @@ def _sig_tier():
     LIB.hga_gather_history.argtypes = [P, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, u32,
                                        vp, vp]
     LIB.hga_install_group_cache.argtypes = [P, i64, vp, C, vp]
-    for n in ("hga_fetch_group_summaries", "hga_gather_history", "hga_install_group_cache"):
+    LIB.hga_gather_history_noalloc.argtypes = [P, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp,
+                                               vp, vp]
+    for n in ("hga_fetch_group_summaries", "hga_gather_history", "hga_install_group_cache",
+              "hga_gather_history_noalloc"):
         getattr(LIB, n).restype = ctypes.c_int
 
 
@@ -325,6 +329,17 @@ def gather_history(p: Params, q_start: int, n_q: int, t_cap: int, tier: HostTier
         _ptr(group_cnt), _ptr(tier.k_host), _ptr(tier.v_host), _ptr(k_dev), _ptr(v_dev),
         _ptr(tier.gen), ctypes.c_uint32(tier.step), _ptr(tier.bytes), _stream(stream)),
         "hga_gather_history")
+
+
+def gather_history_noalloc(p: Params, q_start: int, n_q: int, t_cap: int, tier: HostTier,
+                           group_idx, group_cnt, k_dev, v_dev, stream=None):
+    """gather_history with the generation stamps held inside the library
+    (no device buffer for them from the caller); tier.gen and tier.step are
+    not used."""
+    _ok(LIB.hga_gather_history_noalloc(
+        ctypes.byref(p.c()), q_start, n_q, t_cap, tier.t_hist, _ptr(group_idx),
+        _ptr(group_cnt), _ptr(tier.k_host), _ptr(tier.v_host), _ptr(k_dev), _ptr(v_dev),
+        _ptr(tier.bytes), _stream(stream)), "hga_gather_history_noalloc")
 
 
 def install_group_cache(p: Params, t_cap: int, tier: HostTier, stream=None):
