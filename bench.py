@@ -15,6 +15,7 @@ Prints one JSON line (rank 0).  N > 1 runs independent replicas, one per GPU
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -269,16 +270,38 @@ def run_hga(args, world, rank, local):
     v = inp.v.to(dev)
     bufs = hga.allocate(p, w.T, w.Tq, device=dev)
     stream = torch.cuda.current_stream()
+    # V storage: fp16 (converted once per token as it is committed; the
+    # segment's own tokens are converted inside every step) or bf16 (each
+    # attention tile is converted on chip)
+    v16 = args.v_storage == "f16"
+    p_att = dataclasses.replace(p, v_f16=True) if v16 else p
+    v_att = torch.empty(v.shape, dtype=torch.float16, device=dev) if v16 else v
     # commit the history once (setup, not timed)
     hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+    if v16:
+        hga.convert_v(p, v, 0, w.q0, v_att)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    calls = ([("convert_v", lambda: hga.convert_v(p, v, w.q0, w.T, v_att))] if v16 else []) + [
+        ("build_summaries",
+         lambda: hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)),
+        ("route_chunks",
+         lambda: hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx,
+                                  bufs.chunk_cnt)),
+        ("route_groups",
+         lambda: hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx,
+                                  bufs.chunk_cnt, bufs.group_idx, bufs.group_cnt)),
+        ("attend",
+         lambda: hga.attend(p_att, q, w.q0, k, v_att, bufs.group_idx, bufs.group_cnt, bufs.o,
+                            bufs.lse)),
+    ]
+    names = [n for n, _ in calls]
 
     def step():
-        hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)
-        hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt)
-        hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt,
-                         bufs.group_idx, bufs.group_cnt)
-        hga.attend(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
+        for _, call in calls:
+            call()
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -287,28 +310,29 @@ def run_hga(args, world, rank, local):
     assert hga.check() == 0
     counts = algorithmic_counts(w, bufs.group_cnt.cpu().numpy())
 
-    # One step captured as a CUDA graph so that the four kernels run back to
-    # back on the device (no host gaps); external event nodes between them
-    # give each kernel's device time.
-    n_kern = 4
+    # Two CUDA graphs of one step.  `whole` has event nodes only at its two
+    # ends: the step time, with the kernels back to back and each launch
+    # overlapping the previous kernel's tail.  `split` has an event node
+    # between every two kernels: the per-kernel device times.
+    n_kern = len(calls)
+    ev_w = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(n_kern + 1)]
-    graph = torch.cuda.CUDAGraph()
+    whole, split = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
     cap = torch.cuda.Stream()
     cap.wait_stream(stream)
     launches_cap0 = hga.launch_count()
     with torch.cuda.stream(cap):
-        with torch.cuda.graph(graph, stream=cap):
-            ev[0].record()
-            hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)
-            ev[1].record()
-            hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt)
-            ev[2].record()
-            hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt,
-                             bufs.group_idx, bufs.group_cnt)
-            ev[3].record()
-            hga.attend(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
-            ev[4].record()
+        with torch.cuda.graph(whole, stream=cap):
+            ev_w[0].record()
+            step()
+            ev_w[1].record()
     launches_per_step = hga.launch_count() - launches_cap0
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(split, stream=cap):
+            ev[0].record()
+            for j, (_, call) in enumerate(calls):
+                call()
+                ev[j + 1].record()
     stream.wait_stream(cap)
     torch.cuda.synchronize()
 
@@ -316,28 +340,40 @@ def run_hga(args, world, rank, local):
         t0 = time.perf_counter()
         while time.perf_counter() - t0 < seconds:
             for _ in range(20):
-                graph.replay()
+                whole.replay()
             torch.cuda.synchronize()
+
+    def cold_l2():
+        # outside the events: evict the step's data, then replace the dirty
+        # lines of the write with clean ones so that no write-back of the
+        # flush lands inside the timed step
+        flush.zero_()
+        torch.sum(flush_rd, 0, out=flush_sink)
 
     clocks = ClockSampler(local)
     clocks.start()
     replay_for(args.clock_window)          # load before the timed region (clock samples)
-    per_kernel = np.zeros((args.steps, n_kern))
+    step_ms = np.zeros(args.steps)
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
     for i in range(args.steps):
-        flush.zero_()                      # cold L2, outside the events
-        graph.replay()
+        cold_l2()
+        whole.replay()
         torch.cuda.synchronize()
-        per_kernel[i] = [ev[j].elapsed_time(ev[j + 1]) for j in range(n_kern)]   # ms
+        step_ms[i] = ev_w[0].elapsed_time(ev_w[1])
     torch.cuda.synchronize()
     barrier(world)
     t_wall = time.perf_counter() - t_wall0
+    per_kernel = np.zeros((args.steps, n_kern))
+    for i in range(args.steps):
+        cold_l2()
+        split.replay()
+        torch.cuda.synchronize()
+        per_kernel[i] = [ev[j].elapsed_time(ev[j + 1]) for j in range(n_kern)]   # ms
     replay_for(args.clock_window)          # load after the timed region
     clk = clocks.stop()
     launches = launches_per_step * args.steps
-    step_ms = per_kernel.sum(axis=1)
     ms_local = float(step_ms.mean())
     ms = max_over_ranks(ms_local, world, dev)
     assert hga.check() == 0
@@ -354,7 +390,9 @@ def run_hga(args, world, rank, local):
         q_d.copy_(q_h, non_blocking=True)
         k[:, w.q0:].copy_(kseg_h, non_blocking=True)
         v[:, w.q0:].copy_(vseg_h, non_blocking=True)
-        hga.forward(p, q_d, w.q0, k, v, bufs)
+        if v16:
+            hga.convert_v(p, v, w.q0, w.T, v_att)
+        hga.forward(p_att, q_d, w.q0, k, v_att, bufs)
         o_h.copy_(bufs.o, non_blocking=True)
 
     for _ in range(2):
@@ -379,15 +417,16 @@ def run_hga(args, world, rank, local):
             print(f"dense comparator failed: {exc}", file=sys.stderr)
 
     peaks, peak_kind = load_peaks()
-    att_ms = float(per_kernel[:, 3].mean())
+    col = {n: j for j, n in enumerate(names)}
+    att_ms = float(per_kernel[:, col["attend"]].mean())
     att_tflops = counts["attn_flops"] / (att_ms * 1e-3) / 1e12
     peak_tf = peaks["bf16_tflops"]
     out = None
     if rank == 0:
         n_tok = w.Tq * world
         value = n_tok / (ms * 1e-3)
-        kernels = {name: round(float(per_kernel[:, j].mean()) * 1e3, 2) for j, name in
-                   enumerate(["build_summaries", "route_chunks", "route_groups", "attend"])}
+        kernels = {name: round(float(per_kernel[:, j].mean()) * 1e3, 2)
+                   for j, name in enumerate(names)}
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -399,13 +438,21 @@ def run_hga(args, world, rank, local):
                                   f"local {w.local}, top {w.top_chunks} chunks / "
                                   f"{w.top_groups} groups",
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "flushed (256 MiB write) before every step, outside the events",
-                       "timing": "each step replays one CUDA graph of the 4 calls; "
-                                 "device time between event nodes around the kernels"},
+                       "l2": "flushed before every step, outside the events: 256 MiB "
+                             "written, then another 256 MiB read (no dirty lines left)",
+                       "v_storage": ("fp16 (history converted at commit; the segment's "
+                                     "V converted inside every step)" if v16 else
+                                     "bf16 (converted per tile on chip)"),
+                       "timing": f"step: one CUDA graph of the {n_kern} calls "
+                                 f"({', '.join(names)}) between two event nodes; "
+                                 "kernel_us: a second graph with an event node between "
+                                 "every two kernels"},
             "kernel_us": kernels,
+            "kernel_sum_us": round(float(per_kernel.sum(axis=1).mean()) * 1e3, 2),
             "attn_tflops": att_tflops,
             "route_tflops": (counts["route_chunk_flops"] + counts["route_group_flops"]) /
-                            (float(per_kernel[:, 1:3].sum(axis=1).mean()) * 1e-3) / 1e12,
+                            (float((per_kernel[:, col["route_chunks"]] + per_kernel[:, col["route_groups"]]).mean())
+                             * 1e-3) / 1e12,
             "density": counts["density"],
             "roofline": {"bound": "tensor", "kernel": "hga_attend",
                          "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
@@ -460,6 +507,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
     ap.add_argument("--workload", default=gi.QWEN3_30B_64K.name, choices=sorted(gi.WORKLOADS))
+    ap.add_argument("--v-storage", default="f16", choices=["f16", "bf16"],
+                    help="V cache type read by the attention (f16: converted once per token)")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

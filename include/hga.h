@@ -30,6 +30,7 @@
  * Layouts (all row-major, element type = params.dtype):
  *   q, o        [n_q][n_q_heads][head_dim]          query i is position q_start+i
  *   k, v        [n_kv_heads][t_cap][head_dim]       token t of head h at (h*t_cap+t)*d
+ *               (v in fp16 when params.v_f16 = 1)
  *   chunk_sum   [n_kv_heads][t_cap/chunk][head_dim]
  *   group_sum   [n_kv_heads][t_cap/group][head_dim]
  *   chunk_idx   [n_kv_heads][n_blocks][cap_c]  int32, cap_c = hga_index_capacity(p,t_cap,0)
@@ -91,6 +92,11 @@ typedef struct hga_params {
   int32_t top_chunks;   /* chunk budget per (block, KV head); <= 0 = all       */
   int32_t top_groups;   /* group budget per (block, KV head); <= 0 = all       */
   int32_t dtype;        /* hga_dtype of q, k, v, o and the summaries          */
+  int32_t v_f16;        /* 0: v in dtype.  1: v holds IEEE fp16 values, the  */
+                        /* type of the attention kernels' P.V operand (fp16  */
+                        /* P, 11 significant bits), so they read V as is     */
+                        /* instead of converting each tile; dtype must be    */
+                        /* HGA_BF16.  hga_convert_v fills such a buffer.     */
 } hga_params;
 
 /* Step 1 (section 2.1, "HGA builds two levels of key summaries from the
@@ -145,6 +151,20 @@ hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start,
                       int64_t n_q, const void* k, const void* v, int64_t t_cap,
                       const int32_t* group_idx, const int32_t* group_cnt,
                       void* o, float* lse, hga_stream_t stream);
+
+/* Writes v_f16[h][t] = fp16(v[h][t]) for every KV head h and token
+ * t_begin <= t < t_end (all head_dim values; same [n_kv_heads][t_cap]
+ * [head_dim] layout), for use with params.v_f16 = 1.  Not a step of the
+ * method: it fixes the storage type of V once per token, when the token is
+ * committed, so that the attention kernels need no per-tile conversion.
+ * bf16 -> fp16 rounds to nearest even; it is exact for 2^-14 <= |v| < 65504
+ * and off by at most 2^-25 below.  A |v| above 65504 (inf included)
+ * becomes inf and sets HGA_ERR_DEVICE_CHECK (read by hga_check).  dtype must
+ * be HGA_BF16 (v_f16 in the params is ignored here); v_f16 may equal v (in
+ * place) but must not otherwise overlap it; 0 <= t_begin <= t_end <= t_cap. */
+hga_status hga_convert_v(const hga_params* p, const void* v, int64_t t_cap,
+                         int64_t t_begin, int64_t t_end, void* v_f16,
+                         hga_stream_t stream);
 
 /* Steps 1-4 in one call for a query segment whose own K/V already sit in
  * k/v at [q_start, q_start+n_q): builds the summaries of the segment's
@@ -255,8 +275,8 @@ int64_t hga_launch_count(void);
 const char* hga_last_cuda_error(void);
 
 /* Self-test of the software 2^x the attention kernel evaluates on the FMA
- * pipe for part of each softmax row (Cody-Waite reduction + degree-4
- * polynomial, relative error below 3e-6 for -125 <= x <= 127; smaller x
+ * pipe for part of each softmax row (Cody-Waite reduction + degree-3
+ * polynomial, relative error below 8e-5 for -125 <= x <= 127; smaller x
  * gives 2^-125).  Device arrays x, y of n floats; y[i] = 2^x[i].  Not part of
  * the method: it lets a test compare the kernel's exponential with exp2f. */
 hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t stream);

@@ -99,7 +99,8 @@ __device__ __forceinline__ void convert_tile_bf16_to_f16(char* tile, int n16, in
 constexpr int kAttRows = 64;      // rows per CTA (4 warps x 16)
 constexpr int kAttTok = 64;       // tokens per K/V tile (8 groups)
 
-template <int D>
+// VF16: V is already fp16 in memory (no per-tile conversion).
+template <int D, bool VF16 = false>
 __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
   extern __shared__ __align__(128) char smem[];
   char* sq = smem;                                  // [64][D] bf16, swizzled
@@ -187,7 +188,8 @@ __global__ void __launch_bounds__(128) attend_mma_kernel(AttendArgs a) {
     const char* tk = sk + (t & 1) * (kAttTok * D * 2);
     const char* tv = sv + (t & 1) * (kAttTok * D * 2);
     // V tile bf16 -> fp16 in place (exact for |v| < 65504; larger is reported)
-    convert_tile_bf16_to_f16(sv + (t & 1) * (kAttTok * D * 2), kAttTok * D / 8, 128);
+    if constexpr (!VF16)
+      convert_tile_bf16_to_f16(sv + (t & 1) * (kAttTok * D * 2), kAttTok * D / 8, 128);
     float s[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)

@@ -19,7 +19,8 @@
 //                 O_i += P_i V    (fp16 P from TMEM x fp16 V, MN-major B)
 //   warps 2-3   convert each V tile bf16 -> fp16 in place (exact below 65504;
 //               P kept in fp16 has 11 significant bits) and zero rows that
-//               hold no attended token
+//               hold no attended token; with V stored as fp16 (VF16) only
+//               the zeroing remains
 //   warps 4-7   softmax of tile Q0, warps 8-11 softmax of tile Q1: one thread
 //               per row reads its S row from TMEM, applies the causal / padding
 //               mask, keeps the running max and sum in fp32, writes P (fp16)
@@ -95,7 +96,84 @@ __device__ __forceinline__ void tl_mark(TlBuf* bf, int kind, int idx) {
 #define HGA_TL(kind, idx) ((void)0)
 #endif
 
+// The MMA issuer (one thread).  Per tile j it issues, for each Q tile i,
+// O_i += P_i(j-1) V(j-1) (once softmax has written P_i(j-1)) and then
+// S_i(j) = Q_i K(j)^T; a last round issues the final P.V.  It is kept out of
+// line so that its loop runs from registers of its own: a descriptor is a
+// 64-bit add per MMA, and the tensor pipe stays fed only if nothing in this
+// loop waits on memory (inlined into the kernel, whose softmax code sets the
+// register allocation, the loop reloaded spilled values per MMA).
+#ifdef HGA_TIMELINE
+struct TlBuf;
+#define HGA_TLI(kind, idx) tl_mark(tlp, kind, idx)
+#else
+#define HGA_TLI(kind, idx) ((void)0)
+#endif
 template <int D>
+__device__ __noinline__ void tc_mma_issuer(TcBars* bars, uint32_t tmem, uint32_t q_base,
+                                          uint32_t slot_base, int nq, int n_tiles,
+                                          volatile int* abort_flag, void* tl) {
+  using L = TcLayout<D>;
+#ifdef HGA_TIMELINE
+  TlBuf* tlp = static_cast<TlBuf*>(tl);
+#else
+  (void)tl;
+#endif
+  constexpr uint32_t kIdS = tc::idesc_f16(kTcRows, kTcTok, 1, 0);
+  constexpr uint32_t kIdPV = tc::idesc_f16(kTcRows, D, 0, 1);
+  bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
+  tc::fence_after_sync();
+  const uint64_t q_desc0 = tc::sdesc_sw128(q_base, 16, 1024);
+  const uint64_t k_desc0 = tc::sdesc_sw128(slot_base, 16, L::kGroupBytes);
+  const uint64_t v_desc0 = tc::sdesc_sw128(slot_base, 1024, L::kGroupBytes);
+  for (int j = 0; ok && j <= n_tiles; ++j) {
+    const bool has_s = j < n_tiles, has_pv = j > 0;
+    const int nk = 2 * j, sk = nk % kTcSlots;
+    const int nv = 2 * j - 1, sv = (nv + kTcSlots) % kTcSlots;
+    if (has_pv && !(ok = tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag))) break;
+    const uint64_t kd = k_desc0 + (uint64_t)((sk * L::kSlotBytes) >> 4);
+    const uint64_t vd = v_desc0 + (uint64_t)((sv * L::kSlotBytes) >> 4);
+    for (int i = 0; i < nq; ++i) {
+      if (has_pv) {
+        if (!(ok = tc::mbar_wait(&bars->p_full[i], (j - 1) & 1, abort_flag))) break;
+        tc::fence_after_sync();
+        const uint32_t acc0 = j == 1 ? 0u : 1u;
+        const uint32_t d_o = tmem + 256 + i * 128, a_p = tmem + i * 128;
+#pragma unroll
+        for (int k = 0; k < kTcTok / 16; ++k)
+          tc::mma_ts(d_o, a_p + k * 8, vd + (uint64_t)((2 * k * L::kGroupBytes) >> 4), kIdPV,
+                     k > 0 ? 1u : acc0);
+        tc::mma_commit(&bars->o_full[i]);
+        HGA_TLI(3, (j - 1) * 2 + i);
+      }
+      if (has_s) {
+        if (i == 0) {
+          if (!(ok = tc::mbar_wait(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
+          tc::fence_after_sync();
+        }
+        const uint64_t qd = q_desc0 + (uint64_t)((i * L::kHalves * L::kHalfBytes) >> 4);
+        const uint32_t d_s = tmem + i * 128;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          tc::mma_ss(d_s, qd + (uint64_t)((((k >> 2) * L::kHalfBytes) + (k & 3) * 32) >> 4),
+                     kd + (uint64_t)((((k >> 2) * 1024) + (k & 3) * 32) >> 4), kIdS, k > 0);
+        tc::mma_commit(&bars->s_full[i]);
+        HGA_TLI(2, j * 2 + i);
+      }
+    }
+    if (!ok) break;
+    if (has_pv) tc::mma_commit(&bars->empty[sv]);
+    if (has_s) tc::mma_commit(&bars->empty[sk]);
+  }
+  // drain: every MMA issued so far has completed before TMEM is freed
+  tc::mma_commit(&bars->done);
+  const uint64_t t0 = tc::globaltimer_ns();
+  while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+  }
+}
+#undef HGA_TLI
+
+template <int D, bool VF16 = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k1,
@@ -179,83 +257,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = tc::idesc_f16(kTcRows, kTcTok, 1, 0);
-      constexpr uint32_t kIdPV = tc::idesc_f16(kTcRows, D, 0, 1);
-      const uint32_t q_base = tc::smem_addr(sQ);
-      bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
-      tc::fence_after_sync();
-      // Descriptors are built once; a k-step only moves the start-address
-      // field (bytes >> 4, compile-time offsets), so the issue loop is a
-      // handful of integer adds per MMA and keeps the tensor pipe fed.
-      const uint64_t q_desc0 = tc::sdesc_sw128(q_base, 16, 1024);
-      const uint64_t slot_desc0 = tc::sdesc_sw128(tc::smem_addr(slot_ptr(0, 0)), 16, L::kGroupBytes);
-      const uint64_t v_desc0 = tc::sdesc_sw128(tc::smem_addr(slot_ptr(0, 0)), 1024, L::kGroupBytes);
-      auto issue_s = [&](int i, int s) {
-        const uint64_t ad = q_desc0 + (uint64_t)((i * L::kHalves * L::kHalfBytes) >> 4);
-        const uint64_t bd = slot_desc0 + (uint64_t)((s * L::kSlotBytes) >> 4);
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          constexpr int unused = 0;
-          (void)unused;
-          tc::mma_ss(tmem + i * 128, ad + (uint64_t)((((k >> 2) * L::kHalfBytes) + (k & 3) * 32) >> 4),
-                     bd + (uint64_t)((((k >> 2) * 1024) + (k & 3) * 32) >> 4), kIdS, k > 0);
-        }
-        tc::mma_commit(&bars->s_full[i]);
-      };
-      auto issue_pv = [&](int i, int s, bool first) {
-        const uint64_t bd = v_desc0 + (uint64_t)((s * L::kSlotBytes) >> 4);
-        const uint32_t acc0 = first ? 0u : 1u;
-#pragma unroll
-        for (int k = 0; k < kTcTok / 16; ++k)
-          tc::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
-                     bd + (uint64_t)((2 * k * L::kGroupBytes) >> 4), kIdPV, k > 0 ? 1u : acc0);
-        tc::mma_commit(&bars->o_full[i]);
-      };
-      // PV of tile jp for every Q tile, then release V_jp's slot
-      auto pv_all = [&](int jp) -> bool {
-        const int nv = 2 * jp + 1, sv = nv % kTcSlots;
-        if (!tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag)) return false;
-        for (int i = 0; i < nq; ++i) {
-          if (!tc::mbar_wait(&bars->p_full[i], jp & 1, abort_flag)) return false;
-          tc::fence_after_sync();
-          issue_pv(i, sv, jp == 0);
-          HGA_TL(3, jp * 2 + i);
-        }
-        tc::mma_commit(&bars->empty[sv]);
-        return true;
-      };
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int nk = 2 * j, sk = nk % kTcSlots;
-        const int nv = 2 * (j - 1) + 1, sv = nv % kTcSlots;
-        if (j > 0 && !(ok = tc::mbar_wait(&bars->v_ready[sv], (nv / kTcSlots) & 1, abort_flag)))
-          break;
-        // Per Q tile: PV(j-1) (needs only P(j-1) and V(j-1)), then S(j)
-        // (needs K(j)); each softmax warpgroup finds its next S while the
-        // other tile's products run.
-        for (int i = 0; i < nq && ok; ++i) {
-          if (j > 0) {
-            if (!(ok = tc::mbar_wait(&bars->p_full[i], (j - 1) & 1, abort_flag))) break;
-            tc::fence_after_sync();
-            issue_pv(i, sv, j - 1 == 0);
-            HGA_TL(3, (j - 1) * 2 + i);
-          }
-          if (i == 0) {
-            if (!(ok = tc::mbar_wait(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
-            tc::fence_after_sync();
-          }
-          issue_s(i, sk);
-          HGA_TL(2, j * 2 + i);
-        }
-        if (!ok) break;
-        if (j > 0) tc::mma_commit(&bars->empty[sv]);
-        tc::mma_commit(&bars->empty[sk]);
-      }
-      if (ok && n_tiles > 0) ok = pv_all(n_tiles - 1);
-      // drain: every MMA issued so far has completed before TMEM is freed
-      tc::mma_commit(&bars->done);
-      const uint64_t t0 = tc::globaltimer_ns();
-      while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
-      }
+#ifdef HGA_TIMELINE
+      void* tl = &s_tl;
+#else
+      void* tl = nullptr;
+#endif
+      tc_mma_issuer<D>(bars, tmem, tc::smem_addr(sQ), tc::smem_addr(slot_ptr(0, 0)), nq, n_tiles,
+                       abort_flag, tl);
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -348,7 +356,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool clean = li0 + kTcGroupsPerTile <= n_list && !any_invalid;
       if (clean) clean = ((int64_t)list[li0 + kTcGroupsPerTile - 1] + 1) * a.group <= T;
       char* base = slot_ptr(s, 0);
-      if (clean) {
+      if (VF16 && clean) {
+        // fp16 V as loaded; nothing to do
+      } else if (clean) {
 #pragma unroll
         for (int q0 = 0; q0 < kChunks; q0 += 64 * 8) {
           uint4 raw[8];
@@ -368,12 +378,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int rr = ((q * 16) % 1024) / 128;
           const int li = li0 + g;
           const int ent = li < n_list ? list[li] : -1;
-          uint4 raw = make_uint4(0, 0, 0, 0);
-          if (ent >= 0 && (int64_t)ent * a.group + rr < T) {
-            raw = *reinterpret_cast<const uint4*>(base + q * 16);
-            cvt4(raw);
+          const bool live = ent >= 0 && (int64_t)ent * a.group + rr < T;
+          if constexpr (VF16) {
+            if (!live) *reinterpret_cast<uint4*>(base + q * 16) = make_uint4(0, 0, 0, 0);
+          } else {
+            uint4 raw = make_uint4(0, 0, 0, 0);
+            if (live) {
+              raw = *reinterpret_cast<const uint4*>(base + q * 16);
+              cvt4(raw);
+            }
+            *reinterpret_cast<uint4*>(base + q * 16) = raw;
           }
-          *reinterpret_cast<uint4*>(base + q * 16) = raw;
         }
       }
       tc::fence_proxy_async_smem();
@@ -417,12 +432,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (c > lim) sr[e * 8 + c] = __float_as_uint(-INFINITY);
         }
       }
-      // 8 independent partial maxima (no 128-long dependency chain)
+      // 8 independent partial maxima (no 128-long dependency chain), two
+      // new columns per three-input max
       float mx8[8];
 #pragma unroll
       for (int x = 0; x < 8; ++x) mx8[x] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < kTcTok; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+      for (int c = 0; c < kTcTok; c += 2)
+        mx8[(c >> 1) & 7] = tc::fmax3(mx8[(c >> 1) & 7], __uint_as_float(sr[c]),
+                                      __uint_as_float(sr[c + 1]));
       float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= a.scale_log2;

@@ -1,4 +1,4 @@
-"""Fits the polynomial behind tc::exp2_fma (tc.cuh): 2^f on [-1/2, 1/2].
+"""Fits the polynomial behind tc::exp2_fma2 (tc.cuh): 2^f on [-1/2, 1/2].
 
 Method: least squares, relative-error weighted, on Chebyshev nodes of the
 interval (a near-minimax fit), for the Cody-Waite style reduction
@@ -29,7 +29,7 @@ def fit(deg: int, n: int = 4000):
 
 
 if __name__ == "__main__":
-    deg = int(sys.argv[1]) if len(sys.argv) > 1 else 4
+    deg = int(sys.argv[1]) if len(sys.argv) > 1 else 3
     c, err = fit(deg)
     print("coefficients:", ", ".join(f"{float(x):.9g}f" for x in c))
     print(f"max relative error (float32 Horner): {err:.3e}")

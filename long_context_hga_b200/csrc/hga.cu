@@ -18,6 +18,7 @@
 #include "route_tc.cuh"
 #include "tier.cuh"
 #include "noalloc.cuh"
+#include "convert_v.cuh"
 
 namespace {
 
@@ -93,6 +94,8 @@ hga_status check_params(const hga_params* p) {
   if (p->chunk % p->group) return HGA_ERR_INVALID_ARG;
   if (p->sink < 0 || p->local < 0 || p->sink % p->chunk || p->local % p->chunk) return HGA_ERR_INVALID_ARG;
   if (p->dtype != HGA_BF16 && p->dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
+  if (p->v_f16 != 0 && p->v_f16 != 1) return HGA_ERR_INVALID_ARG;
+  if (p->v_f16 && p->dtype != HGA_BF16) return HGA_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return HGA_ERR_UNSUPPORTED;
   if (p->chunk != 64 || p->group != 8 || p->qblock != 64) return HGA_ERR_UNSUPPORTED;
   return HGA_OK;
@@ -264,11 +267,11 @@ hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_beg
                     reinterpret_cast<T*>(gs));
 }
 
-template <int D>
+template <int D, bool VF16>
 hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
   using L = hga::TcLayout<D>;
   const size_t smem = L::smem_bytes(a.max_list);
-  hga_status s = allow_smem<hga::attend_tc_kernel<D>>(smem);
+  hga_status s = allow_smem<hga::attend_tc_kernel<D, VF16>>(smem);
   if (s != HGA_OK) return s;
   CUtensorMap tq, tk1, tk8, tv1, tv8;
   const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
@@ -276,7 +279,8 @@ hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
   const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(hga::kTcRows / a.G)};
   if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb)) return HGA_ERR_CUDA;
   // K/V as (64 dims, 8 rows, D/64 halves, group): one box = whole groups
-  // landing as [group][half][8 rows][128 B]
+  // landing as [group][half][8 rows][128 B].  Tiled TMA copies bytes, so the
+  // bf16 map serves fp16 V as well.
   const uint64_t gd[4] = {64, 8, (uint64_t)(D / 64), (uint64_t)a.Hkv * a.t_cap / 8};
   const uint64_t gs[3] = {(uint64_t)D * 2, 128, (uint64_t)D * 2 * 8};
   const uint32_t b1[4] = {64, 8, (uint32_t)(D / 64), 1};
@@ -286,8 +290,8 @@ hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
     return HGA_ERR_CUDA;
   hga::TcArgs ta{a, 2 * hga::kTcRows};
   dim3 grid((a.qblock * a.G + ta.rows_per_cta - 1) / ta.rows_per_cta, a.n_blocks, a.Hkv);
-  return launch_pdl(hga::attend_tc_kernel<D>, grid, dim3(hga::kTcThreads), smem, st, tq, tk1, tk8,
-                    tv1, tv8, ta);
+  return launch_pdl(hga::attend_tc_kernel<D, VF16>, grid, dim3(hga::kTcThreads), smem, st, tq, tk1,
+                    tk8, tv1, tv8, ta);
 }
 
 bool tc_eligible(const hga::AttendArgs& a) {
@@ -298,15 +302,15 @@ bool tc_eligible(const hga::AttendArgs& a) {
          a.n_q < (1ll << 31) && (a.t_cap % a.group) == 0;
 }
 
-template <int D>
+template <int D, bool VF16>
 hga_status launch_attend_bf16(hga::AttendArgs& a, cudaStream_t st) {
   const int variant = g_kernel_variant.load(std::memory_order_relaxed);
-  if (variant != 1 && tc_eligible(a)) return launch_attend_tc<D>(a, st);
+  if (variant != 1 && tc_eligible(a)) return launch_attend_tc<D, VF16>(a, st);
   const size_t smem = hga::attend_mma_smem_bytes<D>(a.max_list);
-  hga_status s = allow_smem<hga::attend_mma_kernel<D>>(smem);
+  hga_status s = allow_smem<hga::attend_mma_kernel<D, VF16>>(smem);
   if (s != HGA_OK) return s;
   dim3 grid((a.qblock * a.G + hga::kAttRows - 1) / hga::kAttRows, a.n_blocks, a.Hkv);
-  return launch_pdl(hga::attend_mma_kernel<D>, grid, dim3(128), smem, st, a);
+  return launch_pdl(hga::attend_mma_kernel<D, VF16>, grid, dim3(128), smem, st, a);
 }
 
 template <int D>
@@ -404,8 +408,12 @@ hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start, int64
   a.max_list = (int)max_list;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->head_dim));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p->dtype == HGA_BF16 && p->v_f16)
+    return p->head_dim == 128 ? launch_attend_bf16<128, true>(a, st)
+                              : launch_attend_bf16<64, true>(a, st);
   if (p->dtype == HGA_BF16)
-    return p->head_dim == 128 ? launch_attend_bf16<128>(a, st) : launch_attend_bf16<64>(a, st);
+    return p->head_dim == 128 ? launch_attend_bf16<128, false>(a, st)
+                              : launch_attend_bf16<64, false>(a, st);
   return p->head_dim == 128 ? launch_attend_f32<128>(a, st) : launch_attend_f32<64>(a, st);
 }
 
@@ -588,6 +596,31 @@ hga_status hga_install_group_cache(const hga_params* p, int64_t t_cap,
                               : go(__nv_bfloat16{}, std::integral_constant<int, 64>{});
   return p->head_dim == 128 ? go(float{}, std::integral_constant<int, 128>{})
                             : go(float{}, std::integral_constant<int, 64>{});
+}
+
+hga_status hga_convert_v(const hga_params* p, const void* v, int64_t t_cap, int64_t t_begin,
+                         int64_t t_end, void* v_f16, hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if (p->dtype != HGA_BF16) return HGA_ERR_INVALID_ARG;
+  if (t_cap <= 0 || t_begin < 0 || t_begin > t_end || t_end > t_cap) return HGA_ERR_INVALID_ARG;
+  if (!v || !v_f16 || ((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(v_f16)) & 15))
+    return HGA_ERR_INVALID_ARG;
+  const char* vb = static_cast<const char*>(v);
+  const char* ob = static_cast<const char*>(v_f16);
+  const int64_t bytes = (int64_t)p->n_kv_heads * t_cap * p->head_dim * 2;
+  if (vb != ob && vb < ob + bytes && ob < vb + bytes) return HGA_ERR_INVALID_ARG;
+  if (t_begin == t_end) return HGA_OK;
+  const int64_t n = (int64_t)p->n_kv_heads * (t_end - t_begin) * (p->head_dim / 8);
+  const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const auto* src = static_cast<const __nv_bfloat16*>(v);
+  auto* dst = static_cast<__half*>(v_f16);
+  return p->head_dim == 128
+             ? launch_pdl(hga::convert_v_kernel<128>, dim3(blocks), dim3(256), 0, st, src, dst,
+                          t_cap, t_begin, t_end, p->n_kv_heads)
+             : launch_pdl(hga::convert_v_kernel<64>, dim3(blocks), dim3(256), 0, st, src, dst,
+                          t_cap, t_begin, t_end, p->n_kv_heads);
 }
 
 hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t stream) {

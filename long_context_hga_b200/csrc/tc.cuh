@@ -211,6 +211,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int ab_bf16, int 
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100 and later).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
@@ -243,10 +250,11 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 // 2^x for a pair of floats on the FMA pipe (to share the load of the MUFU
 // unit).  Cody-Waite reduction (W. J. Cody and W. Waite, "Software Manual for
 // the Elementary Functions", 1980): j = round(x) by adding 1.5 * 2^23, f =
-// x - j in [-1/2, 1/2]; 2^f by a degree-4 polynomial (near-minimax least
+// x - j in [-1/2, 1/2]; 2^f by a degree-3 polynomial (near-minimax least
 // squares on Chebyshev nodes, fitted by csrc/exp2_poly.py, max relative error
-// 2.7e-6 in float32); 2^j added to the exponent field.  x is clamped to
-// >= -125 first (-inf gives 2^-125, which rounds to 0 in fp16).  Valid for
+// 7.8e-5 in float32: a sixth of the fp16 rounding step of P, 2^-11, which is
+// where every result goes); 2^j added to the exponent field.  x is clamped
+// to >= -125 first (-inf gives 2^-125, which rounds to 0 in fp16).  Valid for
 // x <= 127.
 __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
   float x0, x1;
@@ -256,11 +264,10 @@ __device__ __forceinline__ uint64_t exp2_fma2(uint64_t x) {
   const uint64_t t = fadd2(x, magic);                       // j in the low bits
   const uint64_t jj = fadd2(t, pk2(-12582912.f, -12582912.f));
   const uint64_t f = ffma2(jj, pk2(-1.f, -1.f), x);          // x - j
-  uint64_t p = pk2(0.00956051052f, 0.00956051052f);
-  p = ffma2(p, f, pk2(0.0559170395f, 0.0559170395f));
-  p = ffma2(p, f, pk2(0.240249813f, 0.240249813f));
-  p = ffma2(p, f, pk2(0.69312197f, 0.69312197f));
-  p = ffma2(p, f, pk2(0.999999166f, 0.999999166f));
+  uint64_t p = pk2(0.055088684f, 0.055088684f);
+  p = ffma2(p, f, pk2(0.242604047f, 0.242604047f));
+  p = ffma2(p, f, pk2(0.693276227f, 0.693276227f));
+  p = ffma2(p, f, pk2(0.999928951f, 0.999928951f));
   float p0, p1, t0, t1;
   unpk2(p, p0, p1);
   unpk2(t, t0, t1);

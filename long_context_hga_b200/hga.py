@@ -27,7 +27,7 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_launch_count", "hga_last_cuda_error",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
             "hga_gather_history", "hga_install_group_cache",
-            "hga_gather_history_noalloc")
+            "hga_gather_history_noalloc", "hga_convert_v")
 
 
 class HgaError(RuntimeError):
@@ -39,7 +39,7 @@ class HgaError(RuntimeError):
 class CParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "n_q_heads", "n_kv_heads", "head_dim", "chunk", "group", "qblock",
-        "sink", "local", "top_chunks", "top_groups", "dtype")]
+        "sink", "local", "top_chunks", "top_groups", "dtype", "v_f16")]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -56,12 +56,14 @@ class Params:
     top_chunks: int = 4
     top_groups: int = 8
     dtype: str = "bf16"
+    v_f16: bool = False          # v holds fp16 values (see convert_v)
 
     def c(self) -> CParams:
         return CParams(self.n_q_heads, self.n_kv_heads, self.head_dim,
                        self.chunk, self.group, self.qblock, self.sink,
                        self.local, self.top_chunks, self.top_groups,
-                       HGA_BF16 if self.dtype == "bf16" else HGA_FP32)
+                       HGA_BF16 if self.dtype == "bf16" else HGA_FP32,
+                       int(self.v_f16))
 
     @property
     def torch_dtype(self):
@@ -97,6 +99,7 @@ def _load() -> ctypes.CDLL:
         "hga_last_cuda_error": [],
         "hga_set_kernel_variant": [i32],
         "hga_selftest_exp2": [vp, vp, i64, vp],
+        "hga_convert_v": [P, vp, i64, i64, i64, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -184,6 +187,12 @@ def attend(p: Params, q, q_start: int, k, v, group_idx, group_cnt, o,
                        _ptr(k), _ptr(v), k.shape[1], _ptr(group_idx),
                        _ptr(group_cnt), _ptr(o), _ptr(lse), _stream(stream)),
         "hga_attend")
+
+
+def convert_v(p: Params, v, t_begin: int, t_end: int, v_f16, stream=None):
+    """v_f16[:, t_begin:t_end] = fp16(v[:, t_begin:t_end]) (layout [Hkv][t_cap][d])."""
+    _ok(LIB.hga_convert_v(ctypes.byref(p.c()), _ptr(v), v.shape[1], t_begin, t_end,
+                          _ptr(v_f16), _stream(stream)), "hga_convert_v")
 
 
 def forward(p: Params, q, q_start: int, k, v, bufs: "Buffers", stream=None):

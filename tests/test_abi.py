@@ -53,6 +53,12 @@ def test_param_validation(hga):
     bad = ok.c()
     bad.dtype = 7
     assert hga.LIB.hga_validate_params(ctypes.byref(bad)) == hga.HGA_ERR_INVALID_ARG
+    # fp16 V storage: only with bf16 q/k, and the flag is 0 or 1
+    assert hga.validate_params(P(32, 4, 128, v_f16=True)) == 0
+    assert hga.validate_params(P(32, 4, 128, dtype="fp32", v_f16=True)) == hga.HGA_ERR_INVALID_ARG
+    bad = ok.c()
+    bad.v_f16 = 2
+    assert hga.LIB.hga_validate_params(ctypes.byref(bad)) == hga.HGA_ERR_INVALID_ARG
 
 
 def test_index_capacity(hga):
@@ -90,6 +96,16 @@ def test_bad_arguments_rejected_before_launch(hga):
     assert L.hga_build_summaries(pp, fake, 1024, 8, 64, fake, fake, None) == 1
     assert L.hga_build_summaries(pp, fake, 1024, 128, 64, fake, fake, None) == 1
     assert L.hga_build_summaries(pp, fake, 1024, 0, 2048, fake, fake, None) == 1
+    # fp16 V conversion: overlapping (not identical) buffers, unaligned,
+    # reversed range, fp32 params
+    assert L.hga_convert_v(pp, fake, 1024, 0, 64, ctypes.c_void_p(0x1000 + 256), None) == 1
+    assert L.hga_convert_v(pp, ctypes.c_void_p(0x1008), 1024, 0, 64, ctypes.c_void_p(1 << 40),
+                           None) == 1
+    assert L.hga_convert_v(pp, fake, 1024, 64, 0, ctypes.c_void_p(1 << 40), None) == 1
+    p32 = P(8, 2, 128, dtype="fp32").c()
+    assert L.hga_convert_v(ctypes.byref(p32), fake, 1024, 0, 64, ctypes.c_void_p(1 << 40),
+                           None) == 1
+    assert L.hga_convert_v(pp, fake, 1024, 64, 64, ctypes.c_void_p(1 << 40), None) == 0
     # empty work is a no-op, not an error
     assert L.hga_build_summaries(pp, None, 1024, 64, 64, None, None, None) == 0
     assert L.hga_route_chunks(pp, None, 0, 0, None, 1024, None, None, None) == 0
