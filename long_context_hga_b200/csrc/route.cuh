@@ -310,7 +310,9 @@ __device__ void score_f32(const RouteArgs& a, int b, int h, int b0, int nrows,
 
 // Keeps the first k_eff candidates by (score desc, index asc) and writes their
 // ids ascending to out[0..k_eff); `sc` holds the n scores.
-__device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t* out,
+// Radix select reading the scores from shared memory in every pass, for
+// more candidates than the register version holds (portable router only).
+__device__ void select_emit_large(const float* sc, const Cands& cd, int k_eff, int32_t* out,
                             int* hist, int* tmp) {
   const int tid = threadIdx.x;
   const int n = cd.n;
@@ -375,6 +377,135 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
   }
 }
 
+constexpr int kSelPer = 16;   // candidates per thread held in registers (n <= 4096)
+
+__device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t* out,
+                            int* hist, int* tmp) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int n = cd.n;
+  if (k_eff >= n) {
+    for (int i = tid; i < n; i += kRouteThreads) out[i] = cd.id(i);
+    return;
+  }
+  // Thread t owns candidates [t*per, t*per + cnt) and keeps their keys in
+  // registers for every pass (the selection is latency-bound: a dependent
+  // shared-memory load, shuffle or barrier costs tens of cycles here).
+  const int per = (n + kRouteThreads - 1) / kRouteThreads;
+  if (per > kSelPer) {
+    select_emit_large(sc, cd, k_eff, out, hist, tmp);
+    return;
+  }
+  const int i0 = min(n, tid * per), cnt = min(n, i0 + per) - i0;
+  uint32_t kr[kSelPer];
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) kr[e] = e < cnt ? score_key(sc[i0 + e]) : 0u;
+  // ---- radix select of the k-th largest key, most significant bits first.
+  // Bits every key shares (the scores of one block mostly agree in sign and
+  // exponent) need no pass: the first pass starts at the highest bit where
+  // the largest and smallest keys differ.  Each pass: one histogram of an
+  // (up to) 8-bit digit, scanned by warp 0 alone; the histogram is double
+  // buffered so a pass costs two barriers.
+  __shared__ int s_digit, s_above;
+  __shared__ unsigned s_kmax, s_kmin;
+  int* const hb1 = tmp + 32;                     // tmp holds 32 + 256 ints
+  unsigned kmax = 0u, kmin = 0xffffffffu;
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e)
+    if (e < cnt) {
+      kmax = max(kmax, kr[e]);
+      kmin = min(kmin, kr[e]);
+    }
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  if (tid == 0) {
+    s_kmax = 0u;
+    s_kmin = 0xffffffffu;
+  }
+  hist[tid] = 0;
+  hb1[tid] = 0;
+  __syncthreads();
+  if (lane == 0) {
+    atomicMax(&s_kmax, kmax);
+    atomicMin(&s_kmin, kmin);
+  }
+  __syncthreads();
+  const uint32_t diff = s_kmax ^ s_kmin;
+  int top = diff ? 31 - __clz(diff) : -1;          // highest differing bit
+  uint32_t pmask = top < 0 ? 0xffffffffu : (top == 31 ? 0u : ~((2u << top) - 1u));
+  uint32_t prefix = s_kmax & pmask;
+  int k_rem = k_eff;
+  // at most 4 passes (32 bits, <= 8 per pass); unrolled so that each pass's
+  // histogram buffer is known at compile time
+#pragma unroll
+  for (int pass = 0; pass < 4; ++pass) {
+    if (top < 0) break;
+    int* const hcur = (pass & 1) ? hb1 : hist;
+    int* const hnxt = (pass & 1) ? hist : hb1;
+    const int shift = max(0, top - 7);
+    const uint32_t dmask = (2u << (top - shift)) - 1u;   // digit of <= 8 bits
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e)
+      if (e < cnt && (kr[e] & pmask) == prefix) atomicAdd(&hcur[(kr[e] >> shift) & dmask], 1);
+    __syncthreads();
+    if (w == 0) {
+      // lane l covers digits 255-8l .. 248-8l (descending); find the digit
+      // where the count of larger digits first reaches k_rem
+      int c8[8], sum = 0;
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        c8[x] = hcur[255 - 8 * lane - x];
+        sum += c8[x];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = incl - sum;                          // counts of larger digits
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        if (run < k_rem && run + c8[x] >= k_rem) {
+          s_digit = 255 - 8 * lane - x;
+          s_above = run;
+        }
+        run += c8[x];
+      }
+#pragma unroll
+      for (int x = 0; x < 8; ++x) hnxt[8 * lane + x] = 0;   // clear for the next pass
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_digit << shift;
+    pmask |= dmask << shift;
+    k_rem -= s_above;
+    top = shift - 1;
+  }
+  // ---- ordered emission.  One scan of packed counts (keys above the k-th
+  // key, keys equal to it) gives every kept candidate its slot: the larger
+  // keys before it plus the first k_rem equal keys (by position).
+  int n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e)
+    if (e < cnt) {
+      n_gt += kr[e] > prefix;
+      n_eq += kr[e] == prefix;
+    }
+  int tot;
+  const int packed = block_excl_scan((n_gt << 16) | n_eq, tmp, &tot);
+  int gt_before = packed >> 16, eq_before = packed & 0xffff;
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) {
+    if (e >= cnt) break;
+    if (kr[e] > prefix) {
+      out[gt_before + min(eq_before, k_rem)] = cd.id(i0 + e);
+      ++gt_before;
+    } else if (kr[e] == prefix) {
+      if (eq_before < k_rem) out[gt_before + eq_before] = cd.id(i0 + e);
+      ++eq_before;
+    }
+  }
+}
+
 // Kept chunks of (b, h) from the chunk router's output, compacted into smem:
 // entry i is kept when it lies in the candidate window [lo, hi) and exceeds
 // entry i-1 (the list must be strictly ascending).  Anything else is reported
@@ -422,7 +553,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(RouteArgs a) {
   __shared__ int s_kept[2048];
   __shared__ int s_nkept;
   __shared__ int hist[256];
-  __shared__ int tmp[32];
+  __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
 
   // ---- candidates
   Cands cd;

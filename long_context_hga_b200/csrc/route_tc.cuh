@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __shared__ int s_kept[2048];
   __shared__ int s_nkept;
   __shared__ int hist[256];
-  __shared__ int tmp[32];
+  __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 #ifdef HGA_TIMELINE
