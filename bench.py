@@ -287,12 +287,18 @@ def run_hga(args, world, rank, local):
     calls = ([("convert_v", lambda: hga.convert_v(p, v, w.q0, w.T, v_att))] if v16 else []) + [
         ("build_summaries",
          lambda: hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)),
+    ] + ([
+        ("route",
+         lambda: hga.route(p, q, w.q0, bufs.chunk_sum, bufs.group_sum, w.T, bufs.chunk_idx,
+                           bufs.chunk_cnt, bufs.group_idx, bufs.group_cnt)),
+    ] if args.route == "fused" else [
         ("route_chunks",
          lambda: hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx,
                                   bufs.chunk_cnt)),
         ("route_groups",
          lambda: hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx,
                                   bufs.chunk_cnt, bufs.group_idx, bufs.group_cnt)),
+    ]) + [
         ("attend",
          lambda: hga.attend(p_att, q, w.q0, k, v_att, bufs.group_idx, bufs.group_cnt, bufs.o,
                             bufs.lse)),
@@ -451,7 +457,7 @@ def run_hga(args, world, rank, local):
             "kernel_sum_us": round(float(per_kernel.sum(axis=1).mean()) * 1e3, 2),
             "attn_tflops": att_tflops,
             "route_tflops": (counts["route_chunk_flops"] + counts["route_group_flops"]) /
-                            (float((per_kernel[:, col["route_chunks"]] + per_kernel[:, col["route_groups"]]).mean())
+                            (float(sum(per_kernel[:, col[n]] for n in col if n.startswith("route")).mean())
                              * 1e-3) / 1e12,
             "density": counts["density"],
             "roofline": {"bound": "tensor", "kernel": "hga_attend",
@@ -509,6 +515,8 @@ def main():
     ap.add_argument("--workload", default=gi.QWEN3_30B_64K.name, choices=sorted(gi.WORKLOADS))
     ap.add_argument("--v-storage", default="f16", choices=["f16", "bf16"],
                     help="V cache type read by the attention (f16: converted once per token)")
+    ap.add_argument("--route", default="split", choices=["fused", "split"],
+                    help="chunk + group routing in one kernel (fused) or two")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -139,6 +139,22 @@ hga_status hga_route_groups(const hga_params* p, const void* q,
                             int32_t* group_idx, int32_t* group_cnt,
                             hga_stream_t stream);
 
+/* Steps 2 and 3 in one call: the same chunk_idx/chunk_cnt and group_idx/
+ * group_cnt as hga_route_chunks followed by hga_route_groups (bit for bit).
+ * On the tensor-core path one CTA per (query block, KV head) runs both: the
+ * block's rows are staged once and the kept chunks go straight from the
+ * chunk selection into the group scoring.  Otherwise the two calls above are
+ * made in order.  One launch instead of two; on the 64K-context workload the
+ * fused kernel is faster alone but, inside a full step, the two launches
+ * finish sooner (hga_forward uses them).  Arguments, capacities and errors
+ * as for those two calls;
+ * chunk_sum must hold every candidate chunk and group_sum every group of the
+ * candidate chunks. */
+hga_status hga_route(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                     const void* chunk_sum, const void* group_sum, int64_t t_cap,
+                     int32_t* chunk_idx, int32_t* chunk_cnt, int32_t* group_idx,
+                     int32_t* group_cnt, hga_stream_t stream);
+
 /* Step 4 (section 2.1, "Exact-token attention": only exact token K/V, never
  * summaries).  Query at position pos (block start b0, query head hq, KV head
  * h = hq / (n_q_heads/n_kv_heads)) attends the set

@@ -182,6 +182,30 @@ hga_status launch_route_tc(hga::RouteArgs& a, cudaStream_t st) {
                     ts8, ra);
 }
 
+template <int D>
+hga_status launch_route_fused_tc(const hga::RouteArgs& ac, const hga::RouteArgs& ag,
+                                 cudaStream_t st) {
+  using L = hga::RtLayout<D>;
+  hga_status s = allow_smem<hga::route_fused_tc_kernel<D>>(L::kSmem);
+  if (s != HGA_OK) return s;
+  hga::RtFusedArgs fa{ac, ag, std::min(256, 64 * ac.G)};
+  CUtensorMap tq, tc_, tg8;
+  const uint64_t qd[3] = {(uint64_t)D, (uint64_t)ac.Hq, (uint64_t)ac.n_q};
+  const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)ac.Hq * D * 2};
+  const uint32_t qb[3] = {64, (uint32_t)ac.G, (uint32_t)(fa.rs / ac.G)};
+  const uint64_t cd[2] = {(uint64_t)D, (uint64_t)ac.Hkv * ac.n_summ_cap};
+  const uint64_t gd[2] = {(uint64_t)D, (uint64_t)ag.Hkv * ag.n_summ_cap};
+  const uint64_t ss[1] = {(uint64_t)D * 2};
+  const uint32_t cb[2] = {64, (uint32_t)hga::kRtTile};
+  const uint32_t gb[2] = {64, 8};
+  if (!encode_bf16_map(&tq, ac.q, 3, qd, qs, qb) || !encode_bf16_map(&tc_, ac.summ, 2, cd, ss, cb) ||
+      !encode_bf16_map(&tg8, ag.summ, 2, gd, ss, gb))
+    return HGA_ERR_CUDA;
+  dim3 grid(ac.n_blocks, ac.Hkv);
+  return launch_pdl(hga::route_fused_tc_kernel<D>, grid, dim3(hga::kRtThreads), L::kSmem, st, tq,
+                    tc_, tg8, fa);
+}
+
 constexpr int kMaxRouteCands = 16384;
 constexpr int kMaxKeptChunks = 2048;
 
@@ -194,17 +218,18 @@ hga_status launch_route(hga::RouteArgs& a, cudaStream_t st) {
   return launch_pdl(hga::route_kernel<T, D>, grid, dim3(hga::kRouteThreads), smem, st, a);
 }
 
-hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
-                        const void* summ, int64_t t_cap, const int32_t* in_idx,
-                        const int32_t* in_cnt, int32_t* out_idx, int32_t* out_cnt, int group_mode,
-                        cudaStream_t st) {
+// Arguments of one routing step; HGA_OK with a.n_q == 0 means nothing to do.
+hga_status route_args(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                      const void* summ, int64_t t_cap, const int32_t* in_idx,
+                      const int32_t* in_cnt, int32_t* out_idx, int32_t* out_cnt, int group_mode,
+                      hga::RouteArgs& a) {
+  a = hga::RouteArgs{};
   hga_status s = check_params(p);
   if (s != HGA_OK) return s;
   if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
   if (n_q == 0) return HGA_OK;
   if (!q || !summ || !out_idx || !out_cnt || (group_mode && (!in_idx || !in_cnt)))
     return HGA_ERR_INVALID_ARG;
-  hga::RouteArgs a{};
   a.q = q;
   a.q_start = q_start;
   a.n_q = n_q;
@@ -242,6 +267,17 @@ hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int
     if (a.in_cap > kMaxKeptChunks || a.in_cap * per > kMaxRouteCands) return HGA_ERR_UNSUPPORTED;
     a.max_cands = (int)std::max<int64_t>(a.in_cap * per, 1);
   }
+  return HGA_OK;
+}
+
+hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                        const void* summ, int64_t t_cap, const int32_t* in_idx,
+                        const int32_t* in_cnt, int32_t* out_idx, int32_t* out_cnt, int group_mode,
+                        cudaStream_t st) {
+  hga::RouteArgs a;
+  hga_status s = route_args(p, q, q_start, n_q, summ, t_cap, in_idx, in_cnt, out_idx, out_cnt,
+                            group_mode, a);
+  if (s != HGA_OK || n_q == 0) return s;
   if (p->dtype == HGA_BF16) {
     if (g_kernel_variant.load(std::memory_order_relaxed) != 1 && route_tc_eligible(a, q, summ))
       return p->head_dim == 128 ? launch_route_tc<128>(a, st) : launch_route_tc<64>(a, st);
@@ -415,6 +451,31 @@ hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start, int64
     return p->head_dim == 128 ? launch_attend_bf16<128, false>(a, st)
                               : launch_attend_bf16<64, false>(a, st);
   return p->head_dim == 128 ? launch_attend_f32<128>(a, st) : launch_attend_f32<64>(a, st);
+}
+
+hga_status hga_route(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                     const void* chunk_sum, const void* group_sum, int64_t t_cap,
+                     int32_t* chunk_idx, int32_t* chunk_cnt, int32_t* group_idx,
+                     int32_t* group_cnt, hga_stream_t stream) {
+  hga::RouteArgs ac, ag;
+  hga_status s = route_args(p, q, q_start, n_q, chunk_sum, t_cap, nullptr, nullptr, chunk_idx,
+                            chunk_cnt, 0, ac);
+  if (s != HGA_OK) return s;
+  if ((s = route_args(p, q, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+                      group_cnt, 1, ag)) != HGA_OK)
+    return s;
+  if (n_q == 0) return HGA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (p->dtype == HGA_BF16 && g_kernel_variant.load(std::memory_order_relaxed) != 1 &&
+      route_tc_eligible(ac, q, chunk_sum) && route_tc_eligible(ag, q, group_sum) &&
+      ac.out_cap <= 2048)
+    return p->head_dim == 128 ? launch_route_fused_tc<128>(ac, ag, st)
+                              : launch_route_fused_tc<64>(ac, ag, st);
+  s = route_common(p, q, q_start, n_q, chunk_sum, t_cap, nullptr, nullptr, chunk_idx, chunk_cnt,
+                   0, st);
+  if (s != HGA_OK) return s;
+  return route_common(p, q, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+                      group_cnt, 1, st);
 }
 
 hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,

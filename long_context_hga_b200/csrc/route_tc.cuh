@@ -40,7 +40,7 @@ struct RtLayout {
   static constexpr int kStageOff = kQBytes;
   static constexpr int kScoreOff = kStageOff + 2 * kStageBytes;
   static constexpr int kBarOff = kScoreOff + kRtMaxCands * 4;
-  static constexpr size_t kSmem = 1024 + (size_t)kBarOff + 256;
+  static constexpr size_t kSmem = 1024 + (size_t)kBarOff + 256;   // 2 barrier sets
 };
 
 struct RtBars {
@@ -53,6 +53,13 @@ struct RtBars {
 // Debug builds only: per-CTA globaltimer stamps (start, scoring start,
 // scoring end, selection end).
 __device__ unsigned long long g_rt[4 * 4096];
+#define HGA_RT_STAMP(slot)                                                          \
+  do {                                                                              \
+    const int cta_l_ = blockIdx.y * gridDim.x + blockIdx.x;                         \
+    if (threadIdx.x == 0 && cta_l_ < 4096) g_rt[4 * cta_l_ + (slot)] = tc::globaltimer_ns(); \
+  } while (0)
+#else
+#define HGA_RT_STAMP(slot) ((void)0)
 #endif
 
 struct RtArgs {
@@ -60,72 +67,23 @@ struct RtArgs {
   int rs;            // query rows per slice (MMA N): min(256, 64 * G)
 };
 
+// Scores every candidate of `cd` for the unit (block at b0, KV head h):
+// sc[i] = max over the unit's rows of q_row . summary(cd.id(i)).  Warp 0
+// streams the summaries (and Q first when load_q; otherwise Q is already in
+// shared memory), warp 1 issues the MMAs into the double-buffered TMEM
+// accumulator at `tmem`, warps 4-7 reduce each candidate's row maxima.  Uses
+// the barrier set `bars` (initialised here) and ends with a CTA barrier.
 template <int D>
-__global__ void __launch_bounds__(kRtThreads, 1)
-    route_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                    const __grid_constant__ CUtensorMap tm_s,
-                    const __grid_constant__ CUtensorMap tm_s8, RtArgs args) {
+__device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool load_q,
+                         const RouteArgs& a, const Cands& cd, int RS, int nrows, int64_t b0,
+                         int h, char* smem, RtBars* bars, uint32_t tmem, float* sc,
+                         volatile int* abort_flag) {
   using L = RtLayout<D>;
-  const RouteArgs& a = args.r;
-  const int RS = args.rs;
-  extern __shared__ __align__(1024) char smem_raw[];
-  char* smem = reinterpret_cast<char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  RtBars* bars = reinterpret_cast<RtBars*>(smem + L::kBarOff);
-  float* sc = reinterpret_cast<float*>(smem + L::kScoreOff);
-  volatile int* abort_flag = &bars->abort;
-  __shared__ int s_kept[2048];
-  __shared__ int s_nkept;
-  __shared__ int hist[256];
-  __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
-
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-#ifdef HGA_TIMELINE
-  if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096)
-    g_rt[4 * (blockIdx.y * gridDim.x + blockIdx.x)] = tc::globaltimer_ns();
-#endif
-  griddep_wait();
-  const int b = blockIdx.x, h = blockIdx.y;
-  const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
-  const int npos = (int)min((int64_t)a.qblock, a.q_start + a.n_q - b0);
-  const int nrows = npos * a.G;
-
-  // ---- candidates (same rules as route_kernel)
-  Cands cd;
-  cd.kept = nullptr;
-  cd.per = a.chunk / a.group;
-  cd.lo = a.sink / a.chunk;
-  const int64_t hi = b0 - a.local > 0 ? (b0 - a.local) / a.chunk : 0;
-  if (!a.group_mode) {
-    cd.n = hi > cd.lo ? (int)(hi - cd.lo) : 0;
-  } else {
-    cd.n = compact_kept_chunks(a, b, h, cd.lo, hi, s_kept, &s_nkept, tmp) * cd.per;
-    cd.kept = s_kept;
-  }
-  const int k_eff = a.top_k <= 0 ? cd.n : min(a.top_k, cd.n);
-  int32_t* out = a.out_idx + ((int64_t)h * a.n_blocks + b) * a.out_cap;
-  if (k_eff > a.out_cap || cd.n > kRtMaxCands) {
-    if (tid == 0) report(HGA_ERR_DEVICE_CHECK);
-    return;
-  }
-  for (int i = k_eff + tid; i < a.out_cap; i += kRtThreads) out[i] = -1;
-  if (tid == 0) a.out_cnt[(int64_t)h * a.n_blocks + b] = k_eff;
-  if (k_eff == 0) return;
-  if (k_eff >= cd.n) {          // every candidate kept: no scores needed
-    select_emit(sc, cd, k_eff, out, hist, tmp);
-    return;
-  }
-
-  // ---- scoring on the tensor cores
-#ifdef HGA_TIMELINE
-  if (tid == 0 && blockIdx.y * gridDim.x + blockIdx.x < 4096)
-    g_rt[4 * (blockIdx.y * gridDim.x + blockIdx.x) + 1] = tc::globaltimer_ns();
-#endif
   const int n_slices = (nrows + RS - 1) / RS;
   const int n_tiles = (cd.n + kRtTile - 1) / kRtTile;
   const int n_jobs = n_tiles * n_slices;
   if (tid == 0) {
-    bars->abort = 0;
     tc::mbar_init(&bars->q_full, 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->full[s], 1);
@@ -136,14 +94,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     tc::mbar_init(&bars->done, 1);
     tc::fence_mbar_init();
   }
-  if (warp == 1) {
-    tc::tmem_alloc(&bars->tmem_base, 512);
-    tc::tmem_relinquish();
-  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  const uint32_t tmem = bars->tmem_base;
   char* sQ = smem;
   auto stage = [&](int s, int hf) { return smem + L::kStageOff + s * L::kStageBytes + hf * L::kTileHalf; };
 
@@ -154,14 +107,16 @@ __global__ void __launch_bounds__(kRtThreads, 1)
     // half; in group mode each kept chunk's 8 groups are one 8-row box per
     // half (lane e < 16 issues kept chunk e of the tile).
     if (lane == 0) {
-      tc::tma_prefetch_desc(&tm_q);
-      tc::tma_prefetch_desc(&tm_s);
-      const int pos0 = (int)(b0 - a.q_start);
-      tc::mbar_arrive_expect_tx(&bars->q_full, n_slices * L::kHalves * RS * 128);
-      for (int r = 0; r < n_slices; ++r)
-        for (int hf = 0; hf < L::kHalves; ++hf)
-          tc::tma_load_3d(sQ + (r * L::kHalves + hf) * L::kQHalf, &tm_q, hf * 64, h * a.G,
-                          pos0 + r * (RS / a.G), &bars->q_full);
+      tc::tma_prefetch_desc(tm_s);
+      if (load_q) {
+        tc::tma_prefetch_desc(tm_q);
+        const int pos0 = (int)(b0 - a.q_start);
+        tc::mbar_arrive_expect_tx(&bars->q_full, n_slices * L::kHalves * RS * 128);
+        for (int r = 0; r < n_slices; ++r)
+          for (int hf = 0; hf < L::kHalves; ++hf)
+            tc::tma_load_3d(sQ + (r * L::kHalves + hf) * L::kQHalf, tm_q, hf * 64, h * a.G,
+                            pos0 + r * (RS / a.G), &bars->q_full);
+      }
     }
     int pending[2] = {-1, -1};
     const int row_head = (int)((int64_t)h * a.n_summ_cap);
@@ -174,7 +129,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         if (lane == 0) {
           tc::mbar_arrive_expect_tx(&bars->full[s], L::kHalves * L::kTileHalf);
           for (int hf = 0; hf < L::kHalves; ++hf)
-            tc::tma_load_2d(stage(s, hf), &tm_s, hf * 64, row_head + cd.lo + t * kRtTile,
+            tc::tma_load_2d(stage(s, hf), tm_s, hf * 64, row_head + cd.lo + t * kRtTile,
                             &bars->full[s]);
         }
       } else {
@@ -184,7 +139,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         if (lane < n_box) {
           const int row = row_head + cd.kept[t * (kRtTile / 8) + lane] * cd.per;
           for (int hf = 0; hf < L::kHalves; ++hf)
-            tc::tma_load_2d(stage(s, hf) + lane * 1024, &tm_s8, hf * 64, row, &bars->full[s]);
+            tc::tma_load_2d(stage(s, hf) + lane * 1024, tm_s, hf * 64, row, &bars->full[s]);
         }
       }
       pending[s] = u;
@@ -203,7 +158,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
       // ------------------------------------------------------------ MMA
       const uint32_t idesc = tc::idesc_f16(kRtTile, RS, 1, 0);
       const uint32_t q_base = tc::smem_addr(sQ);
-      bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
+      bool ok = !load_q || tc::mbar_wait(&bars->q_full, 0, abort_flag);
       for (int t = 0; ok && t < n_tiles; ++t) {
         const int s = t & 1;
         if (!(ok = tc::mbar_wait(&bars->full[s], (t >> 1) & 1, abort_flag))) break;
@@ -252,7 +207,8 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         tc::tmem_wait_ld();
         if (c0 + 128 <= valid_cols && nld == 4) {
 #pragma unroll
-          for (int x = 0; x < 128; ++x) m4[x & 3] = fmaxf(m4[x & 3], __uint_as_float(v[x]));
+          for (int x = 0; x < 128; x += 2)
+            m4[(x >> 1) & 3] = tc::fmax3(m4[(x >> 1) & 3], __uint_as_float(v[x]), __uint_as_float(v[x + 1]));
         } else {
 #pragma unroll
           for (int x = 0; x < 128; ++x)
@@ -271,20 +227,185 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 1) {
-    tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, 512);
+  tc::fence_after_sync();
+}
+
+// Chunk routing or group routing of one (query block, KV head) unit.
+template <int D>
+__global__ void __launch_bounds__(kRtThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_s,
+                    const __grid_constant__ CUtensorMap tm_s8, RtArgs args) {
+  using L = RtLayout<D>;
+  const RouteArgs& a = args.r;
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* smem = reinterpret_cast<char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  RtBars* bars = reinterpret_cast<RtBars*>(smem + L::kBarOff);
+  float* sc = reinterpret_cast<float*>(smem + L::kScoreOff);
+  volatile int* abort_flag = &bars->abort;
+  __shared__ int s_kept[2048];
+  __shared__ int s_nkept;
+  __shared__ int hist[256];
+  __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  HGA_RT_STAMP(0);
+  griddep_wait();
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
+  const int npos = (int)min((int64_t)a.qblock, a.q_start + a.n_q - b0);
+  const int nrows = npos * a.G;
+
+  // ---- candidates (same rules as route_kernel)
+  Cands cd;
+  cd.kept = nullptr;
+  cd.per = a.chunk / a.group;
+  cd.lo = a.sink / a.chunk;
+  const int64_t hi = b0 - a.local > 0 ? (b0 - a.local) / a.chunk : 0;
+  if (!a.group_mode) {
+    cd.n = hi > cd.lo ? (int)(hi - cd.lo) : 0;
+  } else {
+    cd.n = compact_kept_chunks(a, b, h, cd.lo, hi, s_kept, &s_nkept, tmp) * cd.per;
+    cd.kept = s_kept;
   }
+  const int k_eff = a.top_k <= 0 ? cd.n : min(a.top_k, cd.n);
+  int32_t* out = a.out_idx + ((int64_t)h * a.n_blocks + b) * a.out_cap;
+  if (k_eff > a.out_cap || cd.n > kRtMaxCands) {
+    if (tid == 0) report(HGA_ERR_DEVICE_CHECK);
+    return;
+  }
+  for (int i = k_eff + tid; i < a.out_cap; i += kRtThreads) out[i] = -1;
+  if (tid == 0) a.out_cnt[(int64_t)h * a.n_blocks + b] = k_eff;
+  if (k_eff == 0) return;
+  if (k_eff >= cd.n) {          // every candidate kept: no scores needed
+    select_emit(sc, cd, k_eff, out, hist, tmp);
+    return;
+  }
+
+  // ---- scoring on the tensor cores
+  HGA_RT_STAMP(1);
+  if (tid == 0) bars->abort = 0;
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem_base, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+  rt_score<D>(&tm_q, a.group_mode ? &tm_s8 : &tm_s, true, a, cd, args.rs, nrows, b0, h, smem, bars,
+              tmem, sc, abort_flag);
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
   if (*abort_flag) return;
   griddep_launch();
-#ifdef HGA_TIMELINE
-  const int cta_l = blockIdx.y * gridDim.x + blockIdx.x;
-  if (tid == 0 && cta_l < 4096) g_rt[4 * cta_l + 2] = tc::globaltimer_ns();
-#endif
+  HGA_RT_STAMP(2);
   select_emit(sc, cd, k_eff, out, hist, tmp);
-#ifdef HGA_TIMELINE
-  if (tid == 0 && cta_l < 4096) g_rt[4 * cta_l + 3] = tc::globaltimer_ns();
-#endif
+  HGA_RT_STAMP(3);
+}
+
+struct RtFusedArgs {
+  RouteArgs c;       // chunk routing (chunk summaries)
+  RouteArgs g;       // group routing (group summaries); in_idx/in_cnt unused
+  int rs;
+};
+
+// Chunk routing then group routing of one unit in one CTA: the block's rows
+// are staged once, the kept chunks go from the first selection straight into
+// the second scoring pass, and one TMEM allocation serves both.  Writes the
+// same chunk_idx/chunk_cnt and group_idx/group_cnt as the two-kernel path.
+template <int D>
+__global__ void __launch_bounds__(kRtThreads, 1)
+    route_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_c,
+                          const __grid_constant__ CUtensorMap tm_g8, RtFusedArgs args) {
+  using L = RtLayout<D>;
+  const RouteArgs& ac = args.c;
+  const RouteArgs& ag = args.g;
+  extern __shared__ __align__(1024) char smem_raw[];
+  char* smem = reinterpret_cast<char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  RtBars* bars = reinterpret_cast<RtBars*>(smem + L::kBarOff);      // 2 sets: chunks, groups
+  float* sc = reinterpret_cast<float*>(smem + L::kScoreOff);
+  volatile int* abort_flag = &bars[0].abort;
+  __shared__ int s_kept[2048];
+  __shared__ int hist[256];
+  __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  HGA_RT_STAMP(0);
+  griddep_wait();
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int64_t b0 = ac.q_start + (int64_t)b * ac.qblock;
+  const int npos = (int)min((int64_t)ac.qblock, ac.q_start + ac.n_q - b0);
+  const int nrows = npos * ac.G;
+  const int per = ac.chunk / ac.group;
+
+  // ---- chunk candidates
+  Cands cc;
+  cc.kept = nullptr;
+  cc.per = per;
+  cc.lo = ac.sink / ac.chunk;
+  const int64_t hi = b0 - ac.local > 0 ? (b0 - ac.local) / ac.chunk : 0;
+  cc.n = hi > cc.lo ? (int)(hi - cc.lo) : 0;
+  const int k_c = ac.top_k <= 0 ? cc.n : min(ac.top_k, cc.n);
+  int32_t* out_c = ac.out_idx + ((int64_t)h * ac.n_blocks + b) * ac.out_cap;
+  int32_t* out_g = ag.out_idx + ((int64_t)h * ag.n_blocks + b) * ag.out_cap;
+  const int n_g = k_c * per;
+  const int k_g = ag.top_k <= 0 ? n_g : min(ag.top_k, n_g);
+  if (k_c > ac.out_cap || cc.n > kRtMaxCands || k_c > 2048 || n_g > kRtMaxCands ||
+      k_g > ag.out_cap) {
+    if (tid == 0) report(HGA_ERR_DEVICE_CHECK);
+    return;
+  }
+  for (int i = k_c + tid; i < ac.out_cap; i += kRtThreads) out_c[i] = -1;
+  for (int i = k_g + tid; i < ag.out_cap; i += kRtThreads) out_g[i] = -1;
+  if (tid == 0) {
+    ac.out_cnt[(int64_t)h * ac.n_blocks + b] = k_c;
+    ag.out_cnt[(int64_t)h * ag.n_blocks + b] = k_g;
+  }
+  if (k_c == 0) return;
+  const bool score_c = k_c < cc.n, score_g = k_g < n_g;
+
+  if (tid == 0) bars[0].abort = 0;
+  if (score_c || score_g) {
+    if (warp == 1) {
+      tc::tmem_alloc(&bars[0].tmem_base, 512);
+      tc::tmem_relinquish();
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars[0].tmem_base;
+  // ---- chunk scores and selection
+  HGA_RT_STAMP(1);
+  if (score_c)
+    rt_score<D>(&tm_q, &tm_c, true, ac, cc, args.rs, nrows, b0, h, smem, &bars[0], tmem, sc,
+                abort_flag);
+  if (*abort_flag) {
+    if ((score_c || score_g) && warp == 1) tc::tmem_dealloc(tmem, 512);
+    return;
+  }
+  select_emit(sc, cc, k_c, out_c, hist, tmp);
+  __syncthreads();                       // this CTA's chunk_idx writes are visible to it
+  // ---- the kept chunks' groups: scores and selection
+  for (int i = tid; i < k_c; i += kRtThreads) s_kept[i] = out_c[i];
+  __syncthreads();
+  Cands cg;
+  cg.kept = s_kept;
+  cg.per = per;
+  cg.lo = cc.lo;
+  cg.n = n_g;
+  if (score_g)
+    rt_score<D>(&tm_q, &tm_g8, !score_c, ag, cg, args.rs, nrows, b0, h, smem, &bars[1], tmem, sc,
+                abort_flag);
+  if ((score_c || score_g) && warp == 1) tc::tmem_dealloc(tmem, 512);
+  if (*abort_flag) return;
+  griddep_launch();
+  HGA_RT_STAMP(2);
+  select_emit(sc, cg, k_g, out_g, hist, tmp);
+  HGA_RT_STAMP(3);
 }
 
 }  // namespace hga

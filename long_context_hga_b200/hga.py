@@ -27,7 +27,7 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_launch_count", "hga_last_cuda_error",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
             "hga_gather_history", "hga_install_group_cache",
-            "hga_gather_history_noalloc", "hga_convert_v")
+            "hga_gather_history_noalloc", "hga_convert_v", "hga_route")
 
 
 class HgaError(RuntimeError):
@@ -100,6 +100,7 @@ def _load() -> ctypes.CDLL:
         "hga_set_kernel_variant": [i32],
         "hga_selftest_exp2": [vp, vp, i64, vp],
         "hga_convert_v": [P, vp, i64, i64, i64, vp, vp],
+        "hga_route": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -179,6 +180,15 @@ def route_groups(p: Params, q, q_start: int, group_sum, t_cap: int, chunk_idx,
                              _ptr(group_sum), t_cap, _ptr(chunk_idx),
                              _ptr(chunk_cnt), _ptr(group_idx), _ptr(group_cnt),
                              _stream(stream)), "hga_route_groups")
+
+
+def route(p: Params, q, q_start: int, chunk_sum, group_sum, t_cap: int, chunk_idx, chunk_cnt,
+          group_idx, group_cnt, stream=None):
+    """Chunk then group routing in one call (same outputs as route_chunks +
+    route_groups)."""
+    _ok(LIB.hga_route(ctypes.byref(p.c()), _ptr(q), q_start, q.shape[0], _ptr(chunk_sum),
+                      _ptr(group_sum), t_cap, _ptr(chunk_idx), _ptr(chunk_cnt),
+                      _ptr(group_idx), _ptr(group_cnt), _stream(stream)), "hga_route")
 
 
 def attend(p: Params, q, q_start: int, k, v, group_idx, group_cnt, o,

@@ -171,3 +171,33 @@ def test_software_exp2_matches_cuda_exp2f():
     assert rel < 8e-5, rel
     z = hga.selftest_exp2(torch.tensor([-float("inf"), -1e30, -200.0], device="cuda"))
     assert (z >= 0).all() and (z < 3e-38).all()
+
+
+@pytest.mark.parametrize("case", ["30b_64k", "8b_ragged", "g16", "d64_g1", "budget_all", "tiny_fp32"])
+def test_fused_route_equals_two_calls(case):
+    """hga_route (chunk and group routing in one CTA per unit) writes exactly
+    what hga_route_chunks followed by hga_route_groups write."""
+    from long_context_hga_b200 import hga
+    w = {"30b_64k": gi.QWEN3_30B_64K,
+         "8b_ragged": gi.QWEN3_8B_16K.with_(T=4136, q0=2048, n_needles=8),
+         "g16": gi.Workload("g16", 16, 1, 128, 1600, 1024, 1e6, 128, 128, 5, 12, n_needles=4),
+         "d64_g1": gi.Workload("d64_g1", 4, 4, 64, 1536, 512, 1e6, 64, 128, 3, 10, n_needles=4),
+         "budget_all": gi.SWEEP_32K.with_(T=4096, q0=2048, top_chunks=0, top_groups=0),
+         "tiny_fp32": gi.TINY_FP32}[case]
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    dev = torch.device("cuda:0")
+    q, k = inp.q.to(dev), inp.k.to(dev)
+    a = hga.allocate(p, w.T, w.Tq, device=dev)
+    b = hga.allocate(p, w.T, w.Tq, device=dev)
+    hga.build_summaries(p, k, 0, w.T, a.chunk_sum, a.group_sum)
+    hga.route_chunks(p, q, w.q0, a.chunk_sum, w.T, a.chunk_idx, a.chunk_cnt)
+    hga.route_groups(p, q, w.q0, a.group_sum, w.T, a.chunk_idx, a.chunk_cnt, a.group_idx,
+                     a.group_cnt)
+    b.group_idx.fill_(12345)
+    b.chunk_idx.fill_(12345)
+    hga.route(p, q, w.q0, a.chunk_sum, a.group_sum, w.T, b.chunk_idx, b.chunk_cnt, b.group_idx,
+              b.group_cnt)
+    assert hga.check() == 0
+    assert torch.equal(a.chunk_cnt, b.chunk_cnt) and torch.equal(a.chunk_idx, b.chunk_idx)
+    assert torch.equal(a.group_cnt, b.group_cnt) and torch.equal(a.group_idx, b.group_idx)
