@@ -518,6 +518,190 @@ def run_hga(args, world, rank, local):
     return out, w, inp
 
 
+# ---------------------------------------------------------------- other configs
+
+def _time_graph(fn, steps, warmup, flush_w, flush_r, sink):
+    """Device time of fn() as one CUDA graph, cold L2 before each replay."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(g, stream=cap):
+            e0.record()
+            fn()
+            e1.record()
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush_w.zero_()
+        torch.sum(flush_r, 0, out=sink)
+        g.replay()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    del g
+    return float(np.mean(ts))
+
+
+def measure_config(w, args, dev, flush_w, flush_r, sink, dense=True, inp=None):
+    """Whole-step throughput of one workload (inputs resident), with the same
+    step as the headline line: V to fp16 (bf16 workloads), summaries of the
+    segment, chunk and group routing, attention."""
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    inp = inp if inp is not None else gi.make_inputs(w)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    v16 = w.dtype == "bf16"
+    p_att = dataclasses.replace(p, v_f16=True) if v16 else p
+    v_att = torch.empty(v.shape, dtype=torch.float16, device=dev) if v16 else v
+    if w.q0 > 0:
+        hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+        if v16:
+            hga.convert_v(p, v, 0, w.q0, v_att)
+
+    def step():
+        if v16:
+            hga.convert_v(p, v, w.q0, w.T, v_att)
+        hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)
+        hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt)
+        hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt,
+                         bufs.group_idx, bufs.group_cnt)
+        hga.attend(p_att, q, w.q0, k, v_att, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
+
+    ms = _time_graph(step, 10, 3, flush_w, flush_r, sink)
+    assert hga.check() == 0
+    counts = algorithmic_counts(w, bufs.group_cnt.cpu().numpy())
+    peaks, kind = load_peaks()
+    flops = counts["attn_flops"] + counts["route_chunk_flops"] + counts["route_group_flops"]
+    out = {"workload": w.name, "T": w.T, "query_tokens": w.Tq, "dtype": w.dtype,
+           "top_chunks": w.top_chunks, "top_groups": w.top_groups,
+           "ms_per_step": ms, "query_tokens_per_s": w.Tq / (ms * 1e-3),
+           "attended_fraction_of_causal": counts["density"],
+           "step_tflops": flops / (ms * 1e-3) / 1e12,
+           "step_frac_of_tensor_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "peak_source": f"{kind} bf16 burst"}
+    if dense and w.dtype == "bf16":
+        try:
+            dms = dense_sdpa_time(w, q, k, v)
+            out["dense_sdpa"] = {"ms": dms, "query_tokens_per_s": w.Tq / (dms * 1e-3)}
+        except Exception as exc:  # comparator only
+            out["dense_sdpa"] = {"error": str(exc)[:200]}
+    return out, (p, inp, q, k, v, bufs)
+
+
+def dense_reference_fp32(w, q, k, v, rows=1024):
+    """Dense causal attention of the segment in fp32 on the GPU, in slices of
+    query rows (a full score matrix of a 32K prefill would not fit)."""
+    G, d, Hkv = w.G, w.head_dim, w.n_kv_heads
+    out = torch.empty(w.Tq, w.n_q_heads, d, dtype=torch.float32, device=q.device)
+    kf, vf = k[:, :w.T].float(), v[:, :w.T].float()
+    for r0 in range(0, w.Tq, rows):
+        r1 = min(w.Tq, r0 + rows)
+        n, last = r1 - r0, w.q0 + r1                 # keys [0, last)
+        qh = q[r0:r1].float().view(n, Hkv, G, d).permute(1, 2, 0, 3)
+        s = torch.einsum("hgrd,htd->hgrt", qh, kf[:, :last]) / math.sqrt(d)
+        pos = w.q0 + torch.arange(r0, r1, device=q.device)
+        s.masked_fill_(torch.arange(last, device=q.device)[None, :] > pos[:, None], float("-inf"))
+        o = torch.einsum("hgrt,htd->hgrd", torch.softmax(s, dim=-1), vf[:, :last])
+        out[r0:r1] = o.permute(2, 0, 1, 3).reshape(n, w.n_q_heads, d)
+        del s, o
+    return out
+
+
+def measure_tiered(w, dev, flush_w, flush_r, sink, steps=5):
+    """Tiered step of the 128K workload: history K/V and group summaries in
+    pinned host memory, an HBM cache for a quarter of the group summaries,
+    routed history groups gathered over PCIe on a side stream."""
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    q = inp.q.to(dev)
+    full = hga.allocate(p, w.T, w.Tq, device=dev)
+    k_seg = inp.k.to(dev)                      # for the history summaries (commit)
+    hga.build_summaries(p, k_seg, 0, w.q0, full.chunk_sum, full.group_sum)
+    tier = hga.make_host_tier(p, inp.k.pin_memory(), inp.v.pin_memory(),
+                              full.group_sum.cpu().pin_memory(), t_hist=w.q0)
+    del k_seg
+    k_dev = torch.zeros(w.n_kv_heads, w.T, w.head_dim, dtype=torch.bfloat16, device=dev)
+    v_dev = torch.zeros_like(k_dev)
+    k_dev[:, w.q0:] = inp.k[:, w.q0:].to(dev)
+    v_dev[:, w.q0:] = inp.v[:, w.q0:].to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    bufs.chunk_sum.copy_(full.chunk_sum)
+    side = torch.cuda.Stream()
+    hga.tiered_step(p, q, w.q0, tier, k_dev, v_dev, bufs, side)    # cold cache
+    torch.cuda.synchronize()
+    cold = tier.stats.tolist()
+    ts = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0 = int(tier.bytes.item())
+    for _ in range(steps):
+        flush_w.zero_()
+        torch.sum(flush_r, 0, out=sink)
+        e0.record()
+        hga.tiered_step(p, q, w.q0, tier, k_dev, v_dev, bufs, side)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    assert hga.check() == 0
+    warm = (tier.stats - torch.tensor(cold, device=tier.stats.device)).tolist()
+    ms = float(np.mean(ts))
+    return {"workload": w.name, "T": w.T, "query_tokens": w.Tq,
+            "ms_per_step": ms, "query_tokens_per_s": w.Tq / (ms * 1e-3),
+            "timing": "eager tiered_step between CUDA events (host launch gaps included)",
+            "history_on_host": "K/V and group summaries, pinned",
+            "group_cache_slots_fraction": 0.25,
+            "cold_step_hits_misses": cold,
+            "warm_hit_rate": warm[0] / max(1, warm[0] + warm[1]),
+            "pcie_bytes_per_step": (int(tier.bytes.item()) - b0) / steps}
+
+
+def measure_all_configs(args, dev):
+    """Every other workload, briefly (the headline line times the 64K one)."""
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    res = []
+    for w in (gi.TINY_FP32, gi.QWEN3_8B_16K):
+        try:
+            res.append(measure_config(w, args, dev, flush_w, flush_r, sink)[0])
+        except Exception as exc:
+            res.append({"workload": w.name, "error": str(exc)[:300]})
+    try:
+        res.append(measure_tiered(gi.TIERED_128K, dev, flush_w, flush_r, sink))
+    except Exception as exc:
+        res.append({"workload": gi.TIERED_128K.name, "error": str(exc)[:300]})
+    # budget sweep at 32K: sparsity vs throughput vs max error against dense
+    sweep = []
+    dense_o = None
+    sweep_inp = gi.make_inputs(gi.SWEEP_32K)        # the budgets do not change the inputs
+    for kc in gi.SWEEP_BUDGETS:
+        w = gi.SWEEP_32K.with_(top_chunks=kc, top_groups=2 * kc)
+        try:
+            r, (p, inp, q, k, v, bufs) = measure_config(w, args, dev, flush_w, flush_r, sink,
+                                                          dense=dense_o is None, inp=sweep_inp)
+            if dense_o is None:
+                dense_o = dense_reference_fp32(w, q, k, v)
+            err = (bufs.o.float() - dense_o).abs()
+            r["max_abs_err_vs_dense"] = float(err.max())
+            r["mean_abs_err_vs_dense"] = float(err.mean())
+            sweep.append(r)
+            del p, inp, q, k, v, bufs
+        except Exception as exc:
+            sweep.append({"workload": w.name, "top_chunks": kc, "error": str(exc)[:300]})
+    res.append({"workload": gi.SWEEP_32K.name, "budget_sweep": sweep})
+    del flush_w, flush_r
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_reference(args, world, rank):
     """The oracle as the reference arm: CPU, host cores, bounded sample."""
     if rank != 0:
@@ -555,6 +739,8 @@ def main():
     ap.add_argument("--route", default="split", choices=["fused", "split"],
                     help="chunk + group routing in one kernel (fused) or two")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the brief per-workload report of the other configurations")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--clock-window", type=float, default=0.6,
@@ -570,6 +756,8 @@ def main():
         out, w, inp = run_hga(args, world, rank, local)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_seconds)
+        if rank == 0 and world == 1 and not args.no_configs:
+            out["configs"] = measure_all_configs(args, torch.device("cuda", local))
     if out is not None:
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -67,6 +67,7 @@ struct TcLayout {
 struct TcBars {
   uint64_t q_full, full[kTcSlots], empty[kTcSlots], v_ready[kTcSlots];
   uint64_t s_full[2], p_full[2], o_full[2], done;
+  uint64_t ostage[2];    // per Q tile: all rows of O staged in shared memory
   uint32_t tmem_base;
   int abort;
 };
@@ -179,7 +180,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      const __grid_constant__ CUtensorMap tm_k1,
                      const __grid_constant__ CUtensorMap tm_k8,
                      const __grid_constant__ CUtensorMap tm_v1,
-                     const __grid_constant__ CUtensorMap tm_v8, TcArgs args) {
+                     const __grid_constant__ CUtensorMap tm_v8,
+                     const __grid_constant__ CUtensorMap tm_o, TcArgs args) {
   using L = TcLayout<D>;
   const AttendArgs& a = args.a;
   extern __shared__ __align__(1024) char smem_raw[];
@@ -235,6 +237,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::mbar_init(&bars->o_full[i], 1);
     }
     tc::mbar_init(&bars->done, 1);
+    tc::mbar_init(&bars->ostage[0], kTcRows);
+    tc::mbar_init(&bars->ostage[1], kTcRows);
     tc::fence_mbar_init();
   }
   if (warp == 1) {
@@ -526,31 +530,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (tid == 128 || tid == 256) HGA_TL(8, i);
       const float inv_l = 1.f / l;
       bool nonfinite = false;   // inf/NaN output: V outside the fp16 range (or bad input)
-      __nv_bfloat16* dst = nullptr;
-      if (row_live)
-        dst = reinterpret_cast<__nv_bfloat16*>(a.o) +
-              ((pos - a.q_start) * a.Hq + (int64_t)h * a.G + unit_row % a.G) * D;
+      // O / l as bf16 into this Q tile's shared memory (free once its last
+      // S product completed, which o_full implies), in the layout the Q load
+      // used: [half][row][128 B], 128-byte swizzle; one thread then stores the
+      // tile with TMA.  The store box holds at most one query block's
+      // positions, and rows past the segment fall outside the tensor, so only
+      // this unit's rows are written.
+      char* stage = sQ + i * L::kHalves * L::kHalfBytes;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
         tc::tmem_ld32(t_o + c * 32, orr);
         tc::tmem_wait_ld();
-        if (row_live) {
 #pragma unroll
-          for (int q = 0; q < 32; q += 8) {
-            uint4 pk4;
-            uint32_t* pw = reinterpret_cast<uint32_t*>(&pk4);
+        for (int q8 = 0; q8 < 4; ++q8) {
+          uint4 pk4;
+          uint32_t* pw = reinterpret_cast<uint32_t*>(&pk4);
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float o0 = __uint_as_float(orr[q + 2 * t]) * inv_l;
-              const float o1 = __uint_as_float(orr[q + 2 * t + 1]) * inv_l;
-              nonfinite |= !(fabsf(o0) <= 3.0e38f) | !(fabsf(o1) <= 3.0e38f);
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
-              pw[t] = *reinterpret_cast<uint32_t*>(&v2);
-            }
-            *reinterpret_cast<uint4*>(dst + c * 32 + q) = pk4;
+          for (int t = 0; t < 4; ++t) {
+            const float o0 = __uint_as_float(orr[q8 * 8 + 2 * t]) * inv_l;
+            const float o1 = __uint_as_float(orr[q8 * 8 + 2 * t + 1]) * inv_l;
+            nonfinite |= !(fabsf(o0) <= 3.0e38f) | !(fabsf(o1) <= 3.0e38f);
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
+            pw[t] = *reinterpret_cast<uint32_t*>(&v2);
           }
+          const int hf = (c * 32) / 64, ch = ((c * 32) % 64) / 8 + q8;   // 16-byte chunk of the row
+          *reinterpret_cast<uint4*>(stage + hf * L::kHalfBytes + r * 128 + ((ch ^ (r & 7)) * 16)) = pk4;
         }
+      }
+      tc::fence_proxy_async_smem();
+      tc::mbar_arrive(&bars->ostage[i]);
+      if (quarter == 0 && lane == 0 && tc::mbar_wait(&bars->ostage[i], 0, abort_flag)) {
+        const int pos_t = (int)(b0 - a.q_start) + (row0 + i * kTcRows) / a.G;
+#pragma unroll
+        for (int hf = 0; hf < L::kHalves; ++hf)
+          tc::tma_store_3d(&tm_o, hf * 64, h * a.G, pos_t, stage + hf * L::kHalfBytes);
+        tc::bulk_commit_group();
+        tc::bulk_wait_group_read0();
       }
       if (row_live && a.lse)
         a.lse[(pos - a.q_start) * a.Hq + (int64_t)h * a.G + unit_row % a.G] =

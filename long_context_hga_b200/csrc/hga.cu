@@ -309,11 +309,17 @@ hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
   const size_t smem = L::smem_bytes(a.max_list);
   hga_status s = allow_smem<hga::attend_tc_kernel<D, VF16>>(smem);
   if (s != HGA_OK) return s;
-  CUtensorMap tq, tk1, tk8, tv1, tv8;
+  CUtensorMap tq, tk1, tk8, tv1, tv8, to;
   const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
   const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)a.Hq * D * 2};
   const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(hga::kTcRows / a.G)};
-  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb)) return HGA_ERR_CUDA;
+  // O has Q's layout and the epilogue stores a Q tile's rows, but never more
+  // positions than one query block holds: with G = 1 a 128-row tile spans two
+  // blocks, and the second block's rows belong to another CTA.
+  const uint32_t ob[3] = {64, (uint32_t)a.G,
+                          (uint32_t)std::min(hga::kTcRows / a.G, a.qblock)};
+  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb) || !encode_bf16_map(&to, a.o, 3, qd, qs, ob))
+    return HGA_ERR_CUDA;
   // K/V as (64 dims, 8 rows, D/64 halves, group): one box = whole groups
   // landing as [group][half][8 rows][128 B].  Tiled TMA copies bytes, so the
   // bf16 map serves fp16 V as well.
@@ -327,12 +333,12 @@ hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
   hga::TcArgs ta{a, 2 * hga::kTcRows};
   dim3 grid((a.qblock * a.G + ta.rows_per_cta - 1) / ta.rows_per_cta, a.n_blocks, a.Hkv);
   return launch_pdl(hga::attend_tc_kernel<D, VF16>, grid, dim3(hga::kTcThreads), smem, st, tq, tk1,
-                    tk8, tv1, tv8, ta);
+                    tk8, tv1, tv8, to, ta);
 }
 
 bool tc_eligible(const hga::AttendArgs& a) {
   const uintptr_t align = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
-                          reinterpret_cast<uintptr_t>(a.v);
+                          reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.o);
   return (align & 15) == 0 && a.G <= hga::kTcRows && (hga::kTcRows % a.G) == 0 &&
          a.max_list <= hga::kTcMaxList && (int64_t)a.Hkv * a.t_cap < (1ll << 31) &&
          a.n_q < (1ll << 31) && (a.t_cap % a.group) == 0;

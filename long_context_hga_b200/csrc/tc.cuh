@@ -90,6 +90,24 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, int
       "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
       : "memory");
 }
+// 3D tiled store from this CTA's shared memory (bulk group); out-of-bound
+// elements of the box are not written.  Coordinates must be >= 0.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, int x, int y, int z,
+                                             const void* src) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(x), "r"(y), "r"(z), "r"(smem_addr(src))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+}
+// Waits until every committed bulk store of this thread has read its
+// shared-memory source (the stores themselves complete asynchronously).
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, int x, int y, int z,
                                             int w, uint64_t* bar) {
   asm volatile(
