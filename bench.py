@@ -277,16 +277,17 @@ def run_hga(args, world, rank, local):
     p_att = dataclasses.replace(p, v_f16=True) if v16 else p
     v_att = torch.empty(v.shape, dtype=torch.float16, device=dev) if v16 else v
     # commit the history once (setup, not timed)
-    hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
-    if v16:
-        hga.convert_v(p, v, 0, w.q0, v_att)
+    hga.commit(p, k, v, 0, w.q0, bufs.chunk_sum, bufs.group_sum, v_att if v16 else None)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush_sink = torch.empty((), dtype=torch.float32, device=dev)
 
-    calls = ([("convert_v", lambda: hga.convert_v(p, v, w.q0, w.T, v_att))] if v16 else []) + [
-        ("build_summaries",
-         lambda: hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)),
+    # commit of the segment: its summaries and (fp16 V storage) its V in fp16,
+    # one launch
+    calls = [
+        ("commit",
+         lambda: hga.commit(p, k, v, w.q0, w.T, bufs.chunk_sum, bufs.group_sum,
+                            v_att if v16 else None)),
     ] + ([
         ("route",
          lambda: hga.route(p, q, w.q0, bufs.chunk_sum, bufs.group_sum, w.T, bufs.chunk_idx,
@@ -420,9 +421,11 @@ def run_hga(args, world, rank, local):
             s_cmp.wait_event(ev_in[x])
             if i >= 2:
                 s_cmp.wait_event(ev_out[x])         # step i-2's O has been read back
-            if v16:
-                hga.convert_v(p, vb, w.q0, w.T, vab)
-            hga.forward(p_att, q_d, w.q0, kb, vab, bb)
+            hga.commit(p, kb, vb, w.q0, w.T, bb.chunk_sum, bb.group_sum, vab if v16 else None)
+            hga.route_chunks(p, q_d, w.q0, bb.chunk_sum, w.T, bb.chunk_idx, bb.chunk_cnt)
+            hga.route_groups(p, q_d, w.q0, bb.group_sum, w.T, bb.chunk_idx, bb.chunk_cnt,
+                             bb.group_idx, bb.group_cnt)
+            hga.attend(p_att, q_d, w.q0, kb, vab, bb.group_idx, bb.group_cnt, bb.o, bb.lse)
             ev_cmp[x].record(s_cmp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_cmp[x])
@@ -507,7 +510,8 @@ def run_hga(args, world, rank, local):
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "output_matches_device_step": e2e_same,
                     "pipeline": "per step: pinned H2D of Q and the segment's K/V, "
-                                "convert_v + hga_forward, D2H of O; copies on their own "
+                                "commit, route_chunks, route_groups, attend, D2H of O; "
+                                "copies on their own "
                                 "streams overlap the neighbouring steps (2 state sets)"},
             "gpu_launches": int(launches),
             "clocks": clk,
@@ -551,8 +555,8 @@ def _time_graph(fn, steps, warmup, flush_w, flush_r, sink):
 
 def measure_config(w, args, dev, flush_w, flush_r, sink, dense=True, inp=None):
     """Whole-step throughput of one workload (inputs resident), with the same
-    step as the headline line: V to fp16 (bf16 workloads), summaries of the
-    segment, chunk and group routing, attention."""
+    step as the headline line: commit of the segment (summaries, and V to
+    fp16 for bf16 workloads, one launch), chunk and group routing, attention."""
     from long_context_hga_b200 import hga
     p = hga.Params.from_workload(w)
     inp = inp if inp is not None else gi.make_inputs(w)
@@ -562,14 +566,10 @@ def measure_config(w, args, dev, flush_w, flush_r, sink, dense=True, inp=None):
     p_att = dataclasses.replace(p, v_f16=True) if v16 else p
     v_att = torch.empty(v.shape, dtype=torch.float16, device=dev) if v16 else v
     if w.q0 > 0:
-        hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
-        if v16:
-            hga.convert_v(p, v, 0, w.q0, v_att)
+        hga.commit(p, k, v, 0, w.q0, bufs.chunk_sum, bufs.group_sum, v_att if v16 else None)
 
     def step():
-        if v16:
-            hga.convert_v(p, v, w.q0, w.T, v_att)
-        hga.build_summaries(p, k, w.q0, w.T, bufs.chunk_sum, bufs.group_sum)
+        hga.commit(p, k, v, w.q0, w.T, bufs.chunk_sum, bufs.group_sum, v_att if v16 else None)
         hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt)
         hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx, bufs.chunk_cnt,
                          bufs.group_idx, bufs.group_cnt)

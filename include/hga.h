@@ -112,6 +112,22 @@ hga_status hga_build_summaries(const hga_params* p, const void* k,
                                void* chunk_sum, void* group_sum,
                                hga_stream_t stream);
 
+/* Commit of the tokens [t_begin, t_end) in one launch: the summaries of
+ * hga_build_summaries (same arguments, same results) and, when v_f16 is not
+ * NULL, the fp16 copy of V that hga_convert_v writes (v: [Hkv][t_cap][D]
+ * bf16, v_f16: same layout, fp16; every token in [t_begin, t_end), including
+ * a trailing partial chunk).  With v_f16 == NULL it is hga_build_summaries.
+ * The pages have no counterpart; they keep summaries of the projected keys
+ * (section 2.1), and storing V in the attention's operand type when a token
+ * enters the cache is this library's choice.  Requires dtype HGA_BF16 when
+ * v_f16 is given, 16-byte aligned v and v_f16, and v_f16 either equal to v
+ * (in place) or not overlapping it.  A |v| above 65504 becomes inf and sets
+ * HGA_ERR_DEVICE_CHECK (hga_check). */
+hga_status hga_commit(const hga_params* p, const void* k, const void* v,
+                      int64_t t_cap, int64_t t_begin, int64_t t_end,
+                      void* chunk_sum, void* group_sum, void* v_f16,
+                      hga_stream_t stream);
+
 /* Step 2 (section 2.1, "Chunk selection").  For each query block b (queries
  * q_start + b*qblock ...) and KV head h: scores every candidate chunk
  * (sink/chunk <= c < (b0-local)/chunk) by the max over the block's rows of

@@ -289,7 +289,8 @@ hga_status route_common(const hga_params* p, const void* q, int64_t q_start, int
 
 template <typename T, int D>
 hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_begin, int64_t t_end,
-                            int chunk, int group, void* cs, void* gs, cudaStream_t st) {
+                            int chunk, int group, void* cs, void* gs, cudaStream_t st,
+                            const void* v = nullptr, void* v_f16 = nullptr) {
   const int64_t c_first = t_begin / chunk;
   const int64_t c_last = (t_end + chunk - 1) / chunk;   // partial chunk: its closed groups
   const int64_t n_chunks = c_last - c_first;
@@ -300,7 +301,8 @@ hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_beg
   dim3 grid((unsigned)n_chunks, Hkv);
   return launch_pdl(hga::summaries_kernel<T, D>, grid, dim3(32 * hga::kSumGroupsPerChunk), 0, st,
                     reinterpret_cast<const T*>(k), t_cap, c_first, t_end, reinterpret_cast<T*>(cs),
-                    reinterpret_cast<T*>(gs));
+                    reinterpret_cast<T*>(gs), reinterpret_cast<const T*>(v),
+                    reinterpret_cast<__half*>(v_f16));
 }
 
 template <int D, bool VF16>
@@ -399,6 +401,32 @@ hga_status hga_build_summaries(const hga_params* p, const void* k, int64_t t_cap
                                             chunk_sum, group_sum, st)
              : launch_summaries<float, 64>(k, t_cap, Hkv, t_begin, t_end, p->chunk, p->group,
                                            chunk_sum, group_sum, st);
+}
+
+hga_status hga_commit(const hga_params* p, const void* k, const void* v, int64_t t_cap,
+                      int64_t t_begin, int64_t t_end, void* chunk_sum, void* group_sum,
+                      void* v_f16, hga_stream_t stream) {
+  if (!v_f16) return hga_build_summaries(p, k, t_cap, t_begin, t_end, chunk_sum, group_sum, stream);
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if (p->dtype != HGA_BF16) return HGA_ERR_INVALID_ARG;
+  if (t_cap <= 0 || t_begin < 0 || t_begin > t_end || t_end > t_cap) return HGA_ERR_INVALID_ARG;
+  if (t_begin % p->chunk) return HGA_ERR_INVALID_ARG;
+  if (!v || ((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(v_f16)) & 15))
+    return HGA_ERR_INVALID_ARG;
+  const char* vb = static_cast<const char*>(v);
+  const char* ob = static_cast<const char*>(v_f16);
+  const int64_t bytes = (int64_t)p->n_kv_heads * t_cap * p->head_dim * 2;
+  if (vb != ob && vb < ob + bytes && ob < vb + bytes) return HGA_ERR_INVALID_ARG;
+  if (t_begin == t_end) return HGA_OK;
+  if (!k || !chunk_sum || !group_sum) return HGA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int Hkv = p->n_kv_heads;
+  return p->head_dim == 128
+             ? launch_summaries<__nv_bfloat16, 128>(k, t_cap, Hkv, t_begin, t_end, p->chunk,
+                                                    p->group, chunk_sum, group_sum, st, v, v_f16)
+             : launch_summaries<__nv_bfloat16, 64>(k, t_cap, Hkv, t_begin, t_end, p->chunk,
+                                                   p->group, chunk_sum, group_sum, st, v, v_f16);
 }
 
 hga_status hga_route_chunks(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,

@@ -405,7 +405,7 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
   // the largest and smallest keys differ.  Each pass: one histogram of an
   // (up to) 8-bit digit, scanned by warp 0 alone; the histogram is double
   // buffered so a pass costs two barriers.
-  __shared__ int s_digit, s_above;
+  __shared__ int s_digit, s_above, s_in_digit;
   __shared__ unsigned s_kmax, s_kmin;
   int* const hb1 = tmp + 32;                     // tmp holds 32 + 256 ints
   unsigned kmax = 0u, kmin = 0xffffffffu;
@@ -468,6 +468,7 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
         if (run < k_rem && run + c8[x] >= k_rem) {
           s_digit = 255 - 8 * lane - x;
           s_above = run;
+          s_in_digit = c8[x];
         }
         run += c8[x];
       }
@@ -479,16 +480,20 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
     pmask |= dmask << shift;
     k_rem -= s_above;
     top = shift - 1;
+    // every key that shares the resolved prefix is kept: the k-th key need
+    // not be resolved further (the kept set is the same)
+    if (s_in_digit == k_rem) break;
   }
   // ---- ordered emission.  One scan of packed counts (keys above the k-th
-  // key, keys equal to it) gives every kept candidate its slot: the larger
-  // keys before it plus the first k_rem equal keys (by position).
+  // key, keys equal to it, both on the resolved bits pmask) gives every kept
+  // candidate its slot: the larger keys before it plus the first k_rem equal
+  // keys (by position).
   int n_gt = 0, n_eq = 0;
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e)
     if (e < cnt) {
-      n_gt += kr[e] > prefix;
-      n_eq += kr[e] == prefix;
+      n_gt += (kr[e] & pmask) > prefix;
+      n_eq += (kr[e] & pmask) == prefix;
     }
   int tot;
   const int packed = block_excl_scan((n_gt << 16) | n_eq, tmp, &tot);
@@ -496,10 +501,11 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) {
     if (e >= cnt) break;
-    if (kr[e] > prefix) {
+    const uint32_t km = kr[e] & pmask;
+    if (km > prefix) {
       out[gt_before + min(eq_before, k_rem)] = cd.id(i0 + e);
       ++gt_before;
-    } else if (kr[e] == prefix) {
+    } else if (km == prefix) {
       if (eq_before < k_rem) out[gt_before + eq_before] = cd.id(i0 + e);
       ++eq_before;
     }

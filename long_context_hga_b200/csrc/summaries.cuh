@@ -14,6 +14,10 @@
 // sums, staged in shared memory.  HBM-bound: bytes = keys read + summaries
 // written.
 #pragma once
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace hga {
@@ -21,10 +25,16 @@ namespace hga {
 constexpr int kSumGroup = 8;        // tokens per group (validated on the host)
 constexpr int kSumGroupsPerChunk = 8;
 
+// With vout (bf16 keys only), the CTA also stores its chunk's V tokens below
+// t_end as fp16 into vout (same [Hkv][t_cap][D] layout): the commit of a
+// segment in one launch.  Its loads are issued before the key loads so the
+// two round trips overlap.  A magnitude above 65504 becomes inf and raises
+// the device check.
 template <typename T, int D>
 __global__ void __launch_bounds__(32 * kSumGroupsPerChunk) summaries_kernel(
     const T* __restrict__ k, int64_t t_cap, int64_t c_first, int64_t t_end,
-    T* __restrict__ csum, T* __restrict__ gsum) {
+    T* __restrict__ csum, T* __restrict__ gsum, const T* __restrict__ v,
+    __half* __restrict__ vout) {
   constexpr int kVec = Elt<T>::kVec;
   constexpr int kLanesPerRow = D / kVec;          // lanes covering one token row
   constexpr int kRowsPerIter = 32 / kLanesPerRow; // rows per warp load
@@ -43,6 +53,24 @@ __global__ void __launch_bounds__(32 * kSumGroupsPerChunk) summaries_kernel(
   const int col = (lane % kLanesPerRow) * kVec;
   const int sub = lane / kLanesPerRow;
   const T* kh = k + (int64_t)h * t_cap * D;
+
+  // V of this chunk: kChunk rows x D/8 16-byte pieces over the CTA's threads
+  constexpr int kVPieces = kChunk * D / 8;
+  constexpr int kVPer = kVPieces / (32 * kSumGroupsPerChunk);
+  static_assert(kVPieces % (32 * kSumGroupsPerChunk) == 0, "V pieces per thread");
+  uint4 vr[kVPer];
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (vout) {
+#pragma unroll
+      for (int x = 0; x < kVPer; ++x) {
+        const int piece = threadIdx.x + x * 32 * kSumGroupsPerChunk;
+        const int64_t t = c * kChunk + piece / (D / 8);
+        if (t < t_end)
+          vr[x] = __ldg(reinterpret_cast<const uint4*>(v + ((int64_t)h * t_cap + t) * D +
+                                                       (piece % (D / 8)) * 8));
+      }
+    }
+  }
 
   double acc[kVec];
 #pragma unroll
@@ -72,6 +100,28 @@ __global__ void __launch_bounds__(32 * kSumGroupsPerChunk) summaries_kernel(
       }
       *reinterpret_cast<uint4*>(gsum + ((int64_t)h * (t_cap / kSumGroup) + tg / kSumGroup) * D + col) =
           *reinterpret_cast<const uint4*>(out);
+    }
+  }
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    if (vout) {
+      bool overflow = false;
+#pragma unroll
+      for (int x = 0; x < kVPer; ++x) {
+        const int piece = threadIdx.x + x * 32 * kSumGroupsPerChunk;
+        const int64_t t = c * kChunk + piece / (D / 8);
+        if (t >= t_end) continue;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&vr[x]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+          overflow |= (fabsf(f.x) > 65504.f) | (fabsf(f.y) > 65504.f);
+          const __half2 hv = __floats2half2_rn(f.x, f.y);
+          w[j] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(vout + ((int64_t)h * t_cap + t) * D + (piece % (D / 8)) * 8) =
+            vr[x];
+      }
+      if (overflow) report(HGA_ERR_DEVICE_CHECK);
     }
   }
   if (!chunk_closed) return;          // uniform across the CTA

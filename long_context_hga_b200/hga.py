@@ -27,7 +27,7 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_launch_count", "hga_last_cuda_error",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
             "hga_gather_history", "hga_install_group_cache",
-            "hga_gather_history_noalloc", "hga_convert_v", "hga_route")
+            "hga_gather_history_noalloc", "hga_convert_v", "hga_route", "hga_commit")
 
 
 class HgaError(RuntimeError):
@@ -101,6 +101,7 @@ def _load() -> ctypes.CDLL:
         "hga_selftest_exp2": [vp, vp, i64, vp],
         "hga_convert_v": [P, vp, i64, i64, i64, vp, vp],
         "hga_route": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp],
+        "hga_commit": [P, vp, vp, i64, i64, i64, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -203,6 +204,15 @@ def convert_v(p: Params, v, t_begin: int, t_end: int, v_f16, stream=None):
     """v_f16[:, t_begin:t_end] = fp16(v[:, t_begin:t_end]) (layout [Hkv][t_cap][d])."""
     _ok(LIB.hga_convert_v(ctypes.byref(p.c()), _ptr(v), v.shape[1], t_begin, t_end,
                           _ptr(v_f16), _stream(stream)), "hga_convert_v")
+
+
+def commit(p: Params, k, v, t_begin: int, t_end: int, chunk_sum, group_sum, v_f16=None,
+           stream=None):
+    """Summaries of the tokens [t_begin, t_end) (as build_summaries) and, when
+    v_f16 is given, their V in fp16 (as convert_v), in one launch."""
+    _ok(LIB.hga_commit(ctypes.byref(p.c()), _ptr(k), _ptr(v), k.shape[1], t_begin, t_end,
+                       _ptr(chunk_sum), _ptr(group_sum), _ptr(v_f16), _stream(stream)),
+        "hga_commit")
 
 
 def forward(p: Params, q, q_start: int, k, v, bufs: "Buffers", stream=None):

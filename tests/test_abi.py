@@ -106,6 +106,19 @@ def test_bad_arguments_rejected_before_launch(hga):
     assert L.hga_convert_v(ctypes.byref(p32), fake, 1024, 0, 64, ctypes.c_void_p(1 << 40),
                            None) == 1
     assert L.hga_convert_v(pp, fake, 1024, 64, 64, ctypes.c_void_p(1 << 40), None) == 0
+    # segment commit (summaries + fp16 V): overlapping buffers, unaligned V,
+    # fp32 params with a V output, unaligned start, reversed range; without a
+    # V output it is hga_build_summaries
+    out16 = ctypes.c_void_p(1 << 40)
+    assert L.hga_commit(pp, fake, fake, 1024, 0, 64, fake, fake, ctypes.c_void_p(0x1000 + 256),
+                        None) == 1
+    assert L.hga_commit(pp, fake, ctypes.c_void_p(0x1008), 1024, 0, 64, fake, fake, out16,
+                        None) == 1
+    assert L.hga_commit(ctypes.byref(p32), fake, fake, 1024, 0, 64, fake, fake, out16, None) == 1
+    assert L.hga_commit(pp, fake, fake, 1024, 8, 64, fake, fake, out16, None) == 1
+    assert L.hga_commit(pp, fake, fake, 1024, 128, 64, fake, fake, out16, None) == 1
+    assert L.hga_commit(pp, fake, None, 1024, 8, 64, fake, fake, None, None) == 1
+    assert L.hga_commit(pp, fake, fake, 1024, 64, 64, fake, fake, out16, None) == 0
     # empty work is a no-op, not an error
     assert L.hga_build_summaries(pp, None, 1024, 64, 64, None, None, None) == 0
     assert L.hga_route_chunks(pp, None, 0, 0, None, 1024, None, None, None) == 0

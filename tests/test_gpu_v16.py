@@ -61,6 +61,56 @@ def test_convert_v_overflow_sets_device_status():
     assert hga.check() == 0                       # the status word was cleared
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_commit_equals_summaries_and_convert(d):
+    """One launch gives the summaries of build_summaries and the fp16 V of
+    convert_v, bit for bit, over a range that ends in a partial chunk; tokens
+    outside the range keep their bytes; in place works too."""
+    hga = _hga()
+    w = gi.QWEN3_30B_64K.with_(T=1024, q0=0, head_dim=d)
+    p = hga.Params.from_workload(w)
+    g = torch.Generator().manual_seed(11)
+    k = torch.randn(4, 1024, d, generator=g).to(torch.bfloat16).cuda()
+    mag = torch.exp2(torch.randint(-20, 12, (4, 1024, d), generator=g).float())
+    v = (torch.randn(4, 1024, d, generator=g).clamp(-3.9, 3.9) * mag).to(torch.bfloat16).cuda()
+    t0, t1 = 128, 1000                                   # 1000 = 15 chunks + 40 tokens
+    ref_b = hga.allocate(p, 1024, 64, device="cuda")
+    got_b = hga.allocate(p, 1024, 64, device="cuda")
+    for b in (ref_b, got_b):
+        b.chunk_sum.fill_(3.0)
+        b.group_sum.fill_(3.0)
+    ref_v = torch.full(v.shape, 7.0, dtype=torch.float16, device="cuda")
+    got_v = ref_v.clone()
+    hga.build_summaries(p, k, t0, t1, ref_b.chunk_sum, ref_b.group_sum)
+    hga.convert_v(p, v, t0, t1, ref_v)
+    hga.commit(p, k, v, t0, t1, got_b.chunk_sum, got_b.group_sum, got_v)
+    assert hga.check() == 0
+    assert torch.equal(got_b.chunk_sum.view(torch.int16), ref_b.chunk_sum.view(torch.int16))
+    assert torch.equal(got_b.group_sum.view(torch.int16), ref_b.group_sum.view(torch.int16))
+    assert torch.equal(got_v.view(torch.int16), ref_v.view(torch.int16))
+    assert bool((got_v[:, :t0] == 7.0).all()) and bool((got_v[:, t1:] == 7.0).all())
+    inplace = v.clone()
+    hga.commit(p, k, inplace, t0, t1, got_b.chunk_sum, got_b.group_sum, inplace)
+    assert hga.check() == 0
+    assert torch.equal(inplace[:, t0:t1].view(torch.int16), ref_v[:, t0:t1].view(torch.int16))
+    assert torch.equal(inplace[:, :t0], v[:, :t0]) and torch.equal(inplace[:, t1:], v[:, t1:])
+
+
+def test_commit_overflow_sets_device_status():
+    hga = _hga()
+    w = gi.QWEN3_30B_64K.with_(T=256, q0=0)
+    p = hga.Params.from_workload(w)
+    k = torch.zeros(4, 256, 128, dtype=torch.bfloat16, device="cuda")
+    v = torch.zeros(4, 256, 128, dtype=torch.bfloat16, device="cuda")
+    v[2, 200, 7] = -1.0e5
+    b = hga.allocate(p, 256, 64, device="cuda")
+    out = torch.zeros(v.shape, dtype=torch.float16, device="cuda")
+    hga.commit(p, k, v, 0, 256, b.chunk_sum, b.group_sum, out)
+    assert hga.check() == hga.HGA_ERR_DEVICE_CHECK
+    assert torch.isinf(out[2, 200, 7]) and int(torch.isinf(out).sum()) == 1
+    assert hga.check() == 0
+
+
 CASES = {
     "30b_ragged": gi.QWEN3_30B_64K.with_(T=8168, q0=6144, n_needles=16),
     "8b_ragged": gi.QWEN3_8B_16K.with_(T=4136, q0=2048, n_needles=8),
