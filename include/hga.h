@@ -319,9 +319,13 @@ hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t s
  * operands; attention: 128 divisible by the query heads per KV head and at
  * most 4608 attended groups per block; routing: at most 8 query heads per KV
  * head and 4096 candidates per block), 1 = the portable mma.sync kernels,
- * 2 = same as 0.  Both variants compute the same function; tests use the
- * switch to check one against the other.  Returns HGA_ERR_INVALID_ARG for any
- * other value. */
+ * 2 = same as 0, 3 = as 0 but attention with fp16 V and d = 128 runs on CTA
+ * pairs (tcgen05.mma.cta_group::2, M = 256 over two SMs) when a block's rows
+ * fill whole pairs of 256, the query heads per KV head are at least 2 and the
+ * context is a multiple of the group size; it is correct but slower than the
+ * one-CTA kernel on the measured workloads, hence not the default.  All
+ * variants compute the same function; tests use the switch to check one
+ * against another.  Returns HGA_ERR_INVALID_ARG for any other value. */
 hga_status hga_set_kernel_variant(int32_t variant);
 
 #ifdef __cplusplus

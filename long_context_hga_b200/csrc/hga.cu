@@ -15,6 +15,7 @@
 #include "route.cuh"
 #include "attend.cuh"
 #include "attend_tc.cuh"
+#include "attend_pair.cuh"
 #include "route_tc.cuh"
 #include "tier.cuh"
 #include "noalloc.cuh"
@@ -346,9 +347,52 @@ bool tc_eligible(const hga::AttendArgs& a) {
          a.n_q < (1ll << 31) && (a.t_cap % a.group) == 0;
 }
 
+// CTA-pair kernel (d = 128, fp16 V): 256 rows of a unit per pair, so the
+// unit's rows must fill whole pairs; every group in the lists must be whole
+// (context a multiple of the group size), since padding is zero-filled by
+// the loads rather than cleaned up; G >= 2 keeps one CTA's rows inside one
+// query block.
+bool pair_eligible(const hga::AttendArgs& a) {
+  return tc_eligible(a) && a.G >= 2 && ((int64_t)a.qblock * a.G) % 256 == 0 &&
+         ((a.q_start + a.n_q) % a.group) == 0 &&
+         (int64_t)a.Hkv * (a.t_cap / a.group) < (1ll << 31) - 1;
+}
+
+template <int D>
+hga_status launch_attend_pair(hga::AttendArgs& a, cudaStream_t st) {
+  const size_t smem = hga::pair_smem_bytes(a.max_list);
+  hga_status s = allow_smem<hga::attend_pair_kernel<D>>(smem);
+  if (s != HGA_OK) return s;
+  CUtensorMap tq, tk1, tk8, tv1, tv8, to;
+  const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
+  const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)a.Hq * D * 2};
+  const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(hga::kPrRows / a.G)};
+  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb) || !encode_bf16_map(&to, a.o, 3, qd, qs, qb))
+    return HGA_ERR_CUDA;
+  // K/V as (64 dims, 8 rows, D/64 halves, group).  K boxes carry both halves
+  // of a group; V boxes one half (the CTA's), so a V half tile lands as
+  // [group][8 rows][128 B].
+  const uint64_t gd[4] = {64, 8, (uint64_t)(D / 64), (uint64_t)a.Hkv * a.t_cap / 8};
+  const uint64_t gs[3] = {(uint64_t)D * 2, 128, (uint64_t)D * 2 * 8};
+  const uint32_t k1[4] = {64, 8, (uint32_t)(D / 64), 1};
+  const uint32_t k8[4] = {64, 8, (uint32_t)(D / 64), 8};
+  const uint32_t v1[4] = {64, 8, 1, 1};
+  const uint32_t v8[4] = {64, 8, 1, 8};
+  if (!encode_bf16_map(&tk1, a.k, 4, gd, gs, k1) || !encode_bf16_map(&tk8, a.k, 4, gd, gs, k8) ||
+      !encode_bf16_map(&tv1, a.v, 4, gd, gs, v1) || !encode_bf16_map(&tv8, a.v, 4, gd, gs, v8))
+    return HGA_ERR_CUDA;
+  const int pairs = (int)(((int64_t)a.qblock * a.G) / (2 * hga::kPrRows));
+  dim3 grid((unsigned)(2 * pairs), a.n_blocks, a.Hkv);
+  return launch_pdl(hga::attend_pair_kernel<D>, grid, dim3(hga::kPrThreads), smem, st, tq, tk1,
+                    tk8, tv1, tv8, to, a);
+}
+
 template <int D, bool VF16>
 hga_status launch_attend_bf16(hga::AttendArgs& a, cudaStream_t st) {
   const int variant = g_kernel_variant.load(std::memory_order_relaxed);
+  if constexpr (D == 128 && VF16) {
+    if (variant == 3 && pair_eligible(a)) return launch_attend_pair<D>(a, st);
+  }
   if (variant != 1 && tc_eligible(a)) return launch_attend_tc<D, VF16>(a, st);
   const size_t smem = hga::attend_mma_smem_bytes<D>(a.max_list);
   hga_status s = allow_smem<hga::attend_mma_kernel<D, VF16>>(smem);
@@ -571,6 +615,18 @@ int hga_debug_route_times(unsigned long long* out, int max) {
   cudaMemcpyFromSymbol(out, hga::g_rt, n * sizeof(unsigned long long));
   return n;
 }
+int hga_debug_pair_timeline(unsigned long long* out, int max) {
+  cudaDeviceSynchronize();
+  const int n = max < 2 * hga::kPrTlKinds * 128 ? max : 2 * hga::kPrTlKinds * 128;
+  cudaMemcpyFromSymbol(out, hga::g_pr_ev, n * sizeof(unsigned long long));
+  return n;
+}
+int hga_debug_pair_phases(unsigned long long* out, int max) {
+  cudaDeviceSynchronize();
+  const int n = max < 32 ? max : 32;
+  cudaMemcpyFromSymbol(out, hga::g_pr_ph, n * sizeof(unsigned long long));
+  return n;
+}
 int hga_debug_cta_times(unsigned long long* out, int max) {
   cudaDeviceSynchronize();
   const int n = max < 3 * 4096 ? max : 3 * 4096;
@@ -728,7 +784,7 @@ hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t s
 }
 
 hga_status hga_set_kernel_variant(int32_t variant) {
-  if (variant < 0 || variant > 2) return HGA_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 3) return HGA_ERR_INVALID_ARG;
   g_kernel_variant.store(variant, std::memory_order_relaxed);
   return HGA_OK;
 }

@@ -45,11 +45,14 @@ class GpuResult:
 
 
 def run_gpu(w: gi.Workload, inp: gi.Inputs, t_cap: Optional[int] = None,
-            split_history: bool = True) -> GpuResult:
+            split_history: bool = True, v_f16: bool = False) -> GpuResult:
     """History summaries [0, q0) are built first (the committed history), then
-    hga_forward runs summaries of the segment + routing + attention."""
+    hga_forward runs summaries of the segment + routing + attention.  With
+    v_f16 the attention reads V stored as fp16 (converted by the library), as
+    the benchmark does."""
     from long_context_hga_b200 import hga
     p = hga.Params.from_workload(w)
+    p_att = dataclasses.replace(p, v_f16=True) if v_f16 else p
     t_cap = t_cap or w.T
     dev = torch.device("cuda:0")
     q = inp.q.to(dev)
@@ -58,16 +61,20 @@ def run_gpu(w: gi.Workload, inp: gi.Inputs, t_cap: Optional[int] = None,
     k[:, :w.T] = inp.k.to(dev)
     v[:, :w.T] = inp.v.to(dev)
     bufs = hga.allocate(p, t_cap, w.Tq, device=dev)
+    v_att = v
+    if v_f16:
+        v_att = torch.empty(v.shape, dtype=torch.float16, device=dev)
+        hga.convert_v(p, v, 0, t_cap, v_att)
     if split_history and w.q0 > 0:
         hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
-        hga.forward(p, q, w.q0, k, v, bufs)
+        hga.forward(p_att, q, w.q0, k, v_att, bufs)
     else:
         hga.build_summaries(p, k, 0, w.T, bufs.chunk_sum, bufs.group_sum)
         hga.route_chunks(p, q, w.q0, bufs.chunk_sum, t_cap, bufs.chunk_idx,
                          bufs.chunk_cnt)
         hga.route_groups(p, q, w.q0, bufs.group_sum, t_cap, bufs.chunk_idx,
                          bufs.chunk_cnt, bufs.group_idx, bufs.group_cnt)
-        hga.attend(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o,
+        hga.attend(p_att, q, w.q0, k, v_att, bufs.group_idx, bufs.group_cnt, bufs.o,
                    bufs.lse)
     st = hga.check()
     assert st == 0, f"device status {hga.status_string(st)}"

@@ -16,9 +16,9 @@ import parity
 pytestmark = pytest.mark.gpu
 
 
-def _check(w, units=None, split_history=True, t_cap=None):
+def _check(w, units=None, split_history=True, t_cap=None, v_f16=False):
     inp = gi.make_inputs(w)
-    g = parity.run_gpu(w, inp, t_cap=t_cap, split_history=split_history)
+    g = parity.run_gpu(w, inp, t_cap=t_cap, split_history=split_history, v_f16=v_f16)
     rep = parity.compare(w, inp, g, units=units)
     print(w.name, rep)
     assert rep.ok(), rep
@@ -134,14 +134,15 @@ def test_bad_group_index_sets_device_status():
     assert hga.check() == hga.HGA_ERR_DEVICE_CHECK
 
 
+@pytest.mark.parametrize("v_f16", [True, False])
 @pytest.mark.parametrize("name", ["qwen3_30b_a3b_64k_last2k",
                                   "qwen3_8b_prefill_16k"])
-def test_full_size_sampled(name):
-    """Full-size workloads in the benchmark's launch configuration; the
-    oracle recomputes a sample of units."""
+def test_full_size_sampled(name, v_f16):
+    """Full-size workloads; with fp16 V storage this is the benchmark's launch
+    configuration.  The oracle recomputes a sample of units."""
     w = gi.WORKLOADS[name]
     units = parity.sample_units(w, 12)
-    rep, _, _ = _check(w, units=units)
+    rep, _, _ = _check(w, units=units, v_f16=v_f16)
     assert rep.compared_units >= 10
 
 
@@ -155,6 +156,40 @@ def test_attend_variants_agree_with_oracle(variant):
         _check(gi.QWEN3_30B_64K.with_(T=4136, q0=2048, n_needles=8))
     finally:
         hga.set_kernel_variant(0)
+
+
+PAIR_CASES = {
+    "30b_ragged": gi.QWEN3_30B_64K.with_(T=8168, q0=6144, n_needles=16),
+    "8b_g4_ragged": gi.QWEN3_8B_16K.with_(T=2088, n_needles=8),
+    "g16": gi.Workload("g16", 16, 1, 128, 1600, 1024, 1e6, 128, 128, 5, 12, n_needles=4),
+    "budget_all": gi.SWEEP_32K.with_(T=1280, top_chunks=0, top_groups=0, n_needles=4),
+    "short_tail": gi.QWEN3_30B_64K.with_(T=2104, q0=2048, n_needles=4),
+}
+
+
+@pytest.mark.parametrize("case", sorted(PAIR_CASES))
+def test_pair_kernel_agrees_with_oracle_and_single_cta(case):
+    """fp16 V, d = 128: the CTA-pair kernel (variant 3) and the default
+    single-CTA tensor-core kernel both pass the oracle, agree with each other
+    within the output tolerance, and differ in some bits (the pair sums each
+    row's exponentials in two halves, so its kernel really ran)."""
+    from long_context_hga_b200 import hga
+    w = PAIR_CASES[case]
+    inp = gi.make_inputs(w)
+    g_one = parity.run_gpu(w, inp, split_history=w.q0 > 0, v_f16=True)
+    hga.set_kernel_variant(3)
+    try:
+        g_pair = parity.run_gpu(w, inp, split_history=w.q0 > 0, v_f16=True)
+    finally:
+        hga.set_kernel_variant(0)
+    for g in (g_pair, g_one):
+        rep = parity.compare(w, inp, g)
+        print(case, rep)
+        assert rep.ok(), rep
+    assert np.array_equal(g_pair.group_idx, g_one.group_idx)
+    diff = np.abs(g_pair.o - g_one.o)
+    assert float(diff.max()) <= 2e-3 + 1e-2 * float(np.abs(g_one.o).max())
+    assert not np.array_equal(g_pair.o, g_one.o)
 
 
 def test_software_exp2_matches_cuda_exp2f():
