@@ -322,3 +322,63 @@ def dense_causal_attention(q, k, v, q0: int, n_q_heads: int):
         O[:, hq, :] = (e @ v[h]) / z
         L[:, hq] = (m + np.log(z))[:, 0]
     return O, L
+
+
+# ---------------------------------------------------------------- backward
+
+def attend_unit_backward(q, k, v, q0, T, groups: list, p: Params, b: int, h: int,
+                         o, lse, d_o):
+    """Gradients of the exact-token attention of block b, KV head h, with the
+    routed groups held fixed (the selection is piecewise constant, so no
+    gradient flows into the summaries): for a row with attended set R,
+        s_j = q . k_j / sqrt(d),  p_j = exp(s_j - lse),  o = sum_j p_j v_j,
+        dp_j = dO . v_j,  D = dO . o,  ds_j = p_j (dp_j - D),
+        dq = sum_j ds_j k_j / sqrt(d),  dk_j += ds_j q / sqrt(d),  dv_j += p_j dO.
+    o [n_pos][G][d] and lse [n_pos][G] are the forward's outputs as given (the
+    caller's O and LSE, so D and p use the same values a kernel would).
+    Returns (dq [n_pos][G][d], dk [T][d], dv [T][d]) for this unit."""
+    d = q.shape[-1]
+    b0 = q0 + b * p.qblock
+    b1 = min(b0 + p.qblock, T)
+    dq = np.zeros((b1 - b0, p.G, d))
+    dk = np.zeros((T, d))
+    dv = np.zeros((T, d))
+    for pos in range(b0, b1):
+        R = attention_set(b0, pos, groups, p)
+        Kr = k[h, R, :]
+        Vr = v[h, R, :]
+        for gi in range(p.G):
+            qv = q[pos - q0, h * p.G + gi, :]
+            g = d_o[pos - b0, gi]
+            s = Kr @ qv / math.sqrt(d)
+            pj = np.exp(s - lse[pos - b0, gi])
+            dp = Vr @ g
+            D = float(g @ o[pos - b0, gi])
+            ds = pj * (dp - D)
+            dq[pos - b0, gi] = ds @ Kr / math.sqrt(d)
+            dk[R] += np.outer(ds, qv) / math.sqrt(d)
+            dv[R] += np.outer(pj, g)
+    return dq, dk, dv
+
+
+def hga_backward(q, k, v, q0: int, p: Params, group_idx: dict, O, L, dO):
+    """Gradients of the routed attention for the segment [q0, T) with the
+    routing (group lists per (block, KV head)) of a forward pass held fixed.
+    q [Tq][Hq][d], k, v [Hkv][T][d], O and dO [Tq][Hq][d], L [Tq][Hq] (natural
+    log), all float64.  Returns dQ [Tq][Hq][d], dK and dV [Hkv][T][d]."""
+    T = k.shape[1]
+    Tq, Hq, d = q.shape
+    dQ = np.zeros((Tq, Hq, d))
+    dK = np.zeros_like(k)
+    dV = np.zeros_like(v)
+    for h in range(p.n_kv_heads):
+        for b in range(n_blocks(q0, T, p)):
+            r0 = b * p.qblock
+            r1 = min(r0 + p.qblock, Tq)
+            hs = slice(h * p.G, (h + 1) * p.G)
+            dq, dk, dv = attend_unit_backward(q, k, v, q0, T, group_idx[(b, h)], p, b, h,
+                                              O[r0:r1, hs], L[r0:r1, hs], dO[r0:r1, hs])
+            dQ[r0:r1, hs] = dq
+            dK[h] += dk
+            dV[h] += dv
+    return dQ, dK, dV
