@@ -697,9 +697,61 @@ def measure_all_configs(args, dev):
         except Exception as exc:
             sweep.append({"workload": w.name, "top_chunks": kc, "error": str(exc)[:300]})
     res.append({"workload": gi.SWEEP_32K.name, "budget_sweep": sweep})
+    try:
+        res.append(measure_backward(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink))
+    except Exception as exc:
+        res.append({"workload": gi.QWEN3_30B_64K.name, "backward": {"error": str(exc)[:300]}})
     del flush_w, flush_r
     torch.cuda.empty_cache()
     return res
+
+
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1965 MHz
+FP32_ALU_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measure_backward(w, dev, flush_w, flush_r, sink, reps=6):
+    """Backward of the gathered attention (routing of the forward held fixed):
+    device time of hga_attend_backward on the segment with a cold L2, and its
+    algorithmic flops (10 d per (query row, attended token): the S and dP
+    products and the dQ, dK, dV accumulations) against the fp32 peak of the
+    CUDA cores, on which this first version runs."""
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+    hga.forward(p, q, w.q0, k, v, bufs)
+    g = torch.Generator().manual_seed(17)
+    d_o = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+    d_q = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    d_k = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    d_v = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    ts = []
+    for i in range(reps + 2):
+        flush_w.zero_()
+        torch.sum(flush_r, 0, out=sink)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        hga.attend_backward(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse,
+                            d_o, d_q, d_k, d_v)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            ts.append(e0.elapsed_time(e1))
+    assert hga.check() == 0
+    counts = algorithmic_counts(w, bufs.group_cnt.cpu().numpy())
+    flops = counts["attn_flops"] * 10 / 4
+    ms = float(np.median(ts))
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "backward": {
+        "ms": ms, "query_tokens_per_s": w.Tq / (ms * 1e-3),
+        "algorithmic_flops": flops, "tflops": tf,
+        "roofline": {"bound": "alu", "peak": FP32_ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
+                     "frac": tf / FP32_ALU_PEAK_TFLOPS,
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
+        "kernel": "fp32 CUDA cores, one CTA per 128-row slice, 16-byte atomics for dK/dV"}}
 
 
 def run_reference(args, world, rank):

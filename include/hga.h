@@ -184,6 +184,29 @@ hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start,
                       const int32_t* group_idx, const int32_t* group_cnt,
                       void* o, float* lse, hga_stream_t stream);
 
+/* Backward of step 4: gradients of the gathered attention with the routing
+ * held fixed.  The kept groups (group_idx/group_cnt, as used by the forward
+ * pass) are inputs: the selection is piecewise constant, so gradients reach
+ * q, k and v only through the exact-token attention of section 2.1.  For a
+ * query row with attended set R (the same set as hga_attend):
+ *   s_j = q.k_j/sqrt(d), p_j = exp(s_j - lse), dp_j = dO.v_j, D = dO.o,
+ *   ds_j = p_j (dp_j - D); dq = sum_j ds_j k_j/sqrt(d),
+ *   dk_j += ds_j q/sqrt(d), dv_j += p_j dO.
+ * o and lse are the forward's outputs (lse natural log, as hga_attend writes
+ * it); d_o has o's layout and dtype.  Outputs are fp32: d_q [n_q][Hq][d] is
+ * fully written; d_k and d_v [Hkv][t_cap][d] are zeroed on every head's tokens
+ * [0, T) and then accumulated (tokens past T are not touched).  The pages do
+ * not describe a backward; training through the routed attention is how the
+ * paper uses it (section 2.2).  Requires params.v_f16 = 0 (v in dtype),
+ * 16-byte aligned d_q, d_k, d_v; same segment rules as hga_attend.  First
+ * version: fp32 arithmetic on the CUDA cores, atomic adds for d_k and d_v (so
+ * their low bits depend on the order of the adds). */
+hga_status hga_attend_backward(const hga_params* p, const void* q, int64_t q_start,
+                               int64_t n_q, const void* k, const void* v, int64_t t_cap,
+                               const int32_t* group_idx, const int32_t* group_cnt,
+                               const void* o, const float* lse, const void* d_o,
+                               float* d_q, float* d_k, float* d_v, hga_stream_t stream);
+
 /* Writes v_f16[h][t] = fp16(v[h][t]) for every KV head h and token
  * t_begin <= t < t_end (all head_dim values; same [n_kv_heads][t_cap]
  * [head_dim] layout), for use with params.v_f16 = 1.  Not a step of the

@@ -16,6 +16,7 @@
 #include "attend.cuh"
 #include "attend_tc.cuh"
 #include "attend_pair.cuh"
+#include "attend_bwd.cuh"
 #include "route_tc.cuh"
 #include "tier.cuh"
 #include "noalloc.cuh"
@@ -412,6 +413,17 @@ hga_status launch_attend_f32(hga::AttendArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+template <typename T, int D>
+hga_status launch_attend_bwd(hga::BwArgs& w, cudaStream_t st) {
+  using L = hga::BwLayout<D>;
+  const size_t smem = L::smem_bytes(w.a.max_list);
+  hga_status s = allow_smem<hga::attend_bwd_kernel<T, D>>(smem);
+  if (s != HGA_OK) return s;
+  dim3 grid((unsigned)((w.a.qblock * w.a.G + hga::kBwRows - 1) / hga::kBwRows), w.a.n_blocks,
+            w.a.Hkv);
+  return launch_pdl(hga::attend_bwd_kernel<T, D>, grid, dim3(hga::kBwThreads), smem, st, w);
+}
+
 extern "C" {
 
 hga_status hga_validate_params(const hga_params* p) { return check_params(p); }
@@ -529,6 +541,67 @@ hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start, int64
     return p->head_dim == 128 ? launch_attend_bf16<128, false>(a, st)
                               : launch_attend_bf16<64, false>(a, st);
   return p->head_dim == 128 ? launch_attend_f32<128>(a, st) : launch_attend_f32<64>(a, st);
+}
+
+hga_status hga_attend_backward(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                               const void* k, const void* v, int64_t t_cap,
+                               const int32_t* group_idx, const int32_t* group_cnt, const void* o,
+                               const float* lse, const void* d_o, float* d_q, float* d_k,
+                               float* d_v, hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if (p->v_f16) return HGA_ERR_INVALID_ARG;
+  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!q || !k || !v || !group_idx || !group_cnt || !o || !lse || !d_o || !d_q || !d_k || !d_v)
+    return HGA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_q) | reinterpret_cast<uintptr_t>(d_k) |
+       reinterpret_cast<uintptr_t>(d_v)) & 15)
+    return HGA_ERR_INVALID_ARG;
+  hga::BwArgs w{};
+  hga::AttendArgs& a = w.a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q_start = q_start;
+  a.n_q = n_q;
+  a.t_cap = t_cap;
+  a.group_idx = group_idx;
+  a.group_cnt = group_cnt;
+  a.cap_g = cap_groups(p, t_cap);
+  a.n_blocks = (int)((n_q + p->qblock - 1) / p->qblock);
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.G = p->n_q_heads / p->n_kv_heads;
+  a.group = p->group;
+  a.qblock = p->qblock;
+  a.sink = p->sink;
+  a.local = p->local;
+  const int64_t max_list = p->sink / p->group + a.cap_g + p->local / p->group +
+                           (p->qblock + p->group - 1) / p->group;
+  if (max_list > 16384) return HGA_ERR_UNSUPPORTED;
+  a.max_list = (int)max_list;
+  w.o = o;
+  w.d_o = d_o;
+  w.lse = lse;
+  w.d_q = d_q;
+  w.d_k = d_k;
+  w.d_v = d_v;
+  w.scale = (float)(1.0 / sqrt((double)p->head_dim));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // dK and dV are sums over the query rows that attend each token: start
+  // from zero on every head's tokens [0, T)
+  const int64_t T = q_start + n_q;
+  const size_t row_bytes = (size_t)T * p->head_dim * 4;
+  const size_t pitch = (size_t)t_cap * p->head_dim * 4;
+  cudaError_t e = cudaMemset2DAsync(d_k, pitch, 0, row_bytes, p->n_kv_heads, st);
+  if (e == cudaSuccess) e = cudaMemset2DAsync(d_v, pitch, 0, row_bytes, p->n_kv_heads, st);
+  if (e != cudaSuccess) return cuda_ok(e);
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? launch_attend_bwd<__nv_bfloat16, 128>(w, st)
+                              : launch_attend_bwd<__nv_bfloat16, 64>(w, st);
+  return p->head_dim == 128 ? launch_attend_bwd<float, 128>(w, st)
+                            : launch_attend_bwd<float, 64>(w, st);
 }
 
 hga_status hga_route(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,

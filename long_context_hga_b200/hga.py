@@ -27,7 +27,8 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_launch_count", "hga_last_cuda_error",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
             "hga_gather_history", "hga_install_group_cache",
-            "hga_gather_history_noalloc", "hga_convert_v", "hga_route", "hga_commit")
+            "hga_gather_history_noalloc", "hga_convert_v", "hga_route", "hga_commit",
+            "hga_attend_backward")
 
 
 class HgaError(RuntimeError):
@@ -102,6 +103,8 @@ def _load() -> ctypes.CDLL:
         "hga_convert_v": [P, vp, i64, i64, i64, vp, vp],
         "hga_route": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp],
         "hga_commit": [P, vp, vp, i64, i64, i64, vp, vp, vp, vp],
+        "hga_attend_backward": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp,
+                                vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -198,6 +201,17 @@ def attend(p: Params, q, q_start: int, k, v, group_idx, group_cnt, o,
                        _ptr(k), _ptr(v), k.shape[1], _ptr(group_idx),
                        _ptr(group_cnt), _ptr(o), _ptr(lse), _stream(stream)),
         "hga_attend")
+
+
+def attend_backward(p: Params, q, q_start: int, k, v, group_idx, group_cnt, o, lse, d_o,
+                    d_q, d_k, d_v, stream=None):
+    """Gradients of the routed attention with the routing held fixed: d_q
+    [n_q][Hq][d], d_k and d_v [Hkv][t_cap][d] (fp32; d_k/d_v zeroed on the
+    context's tokens, then accumulated)."""
+    _ok(LIB.hga_attend_backward(ctypes.byref(p.c()), _ptr(q), q_start, q.shape[0], _ptr(k),
+                                _ptr(v), k.shape[1], _ptr(group_idx), _ptr(group_cnt),
+                                _ptr(o), _ptr(lse), _ptr(d_o), _ptr(d_q), _ptr(d_k),
+                                _ptr(d_v), _stream(stream)), "hga_attend_backward")
 
 
 def convert_v(p: Params, v, t_begin: int, t_end: int, v_f16, stream=None):

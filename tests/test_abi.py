@@ -119,6 +119,19 @@ def test_bad_arguments_rejected_before_launch(hga):
     assert L.hga_commit(pp, fake, fake, 1024, 128, 64, fake, fake, out16, None) == 1
     assert L.hga_commit(pp, fake, None, 1024, 8, 64, fake, fake, None, None) == 1
     assert L.hga_commit(pp, fake, fake, 1024, 64, 64, fake, fake, out16, None) == 0
+    # backward: V stored as fp16 is not accepted, unaligned or missing outputs
+    p16 = P(8, 2, 128, v_f16=True).c()
+    f32 = ctypes.c_void_p(1 << 40)
+    assert L.hga_attend_backward(ctypes.byref(p16), fake, 0, 64, fake, fake, 1024, fake, fake,
+                                 fake, fake, fake, f32, f32, f32, None) == 1
+    assert L.hga_attend_backward(pp, fake, 0, 64, fake, fake, 1024, fake, fake, fake, fake,
+                                 fake, ctypes.c_void_p((1 << 40) + 4), f32, f32, None) == 1
+    assert L.hga_attend_backward(pp, fake, 0, 64, fake, fake, 1024, fake, fake, fake, None,
+                                 fake, f32, f32, f32, None) == 1
+    assert L.hga_attend_backward(pp, fake, 32, 64, fake, fake, 1024, fake, fake, fake, fake,
+                                 fake, f32, f32, f32, None) == 1
+    assert L.hga_attend_backward(pp, None, 0, 0, None, None, 1024, None, None, None, None,
+                                 None, None, None, None, None) == 0
     # empty work is a no-op, not an error
     assert L.hga_build_summaries(pp, None, 1024, 64, 64, None, None, None) == 0
     assert L.hga_route_chunks(pp, None, 0, 0, None, 1024, None, None, None) == 0
