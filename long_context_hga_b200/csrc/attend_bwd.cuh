@@ -38,7 +38,7 @@ struct BwArgs {
 
 template <int D>
 struct BwLayout {
-  static constexpr int kStride = D + 1;               // padded rows: no bank conflicts
+  static constexpr int kStride = D + 4;   // padded rows, 16-byte aligned: float4 loads without bank conflicts
   static constexpr int kQ = 0;                                        // [128][D+1]
   static constexpr int kDO = kQ + kBwRows * kStride * 4;              // [128][D+1]
   static constexpr int kK = kDO + kBwRows * kStride * 4;              // [8][D+1]
@@ -141,25 +141,32 @@ __global__ void __launch_bounds__(kBwThreads) attend_bwd_kernel(BwArgs w) {
       sv[j * S + c] = in ? bw_load<E>(vh + (t0 + j) * D + c) : 0.f;
     }
     __syncthreads();
-    // ---- p and ds for (row tid/2, tokens 4 (tid%2) .. +4)
+    // ---- p and ds for (row tid/2, tokens 4 (tid%2) .. +4): register tile
+    // of 4 dot products of each kind, 16-byte shared loads along d
     {
       const int r = tid >> 1, j0 = (tid & 1) * 4;
       const int pos = s_pos[r];
+      float sv4[4] = {0.f, 0.f, 0.f, 0.f}, dp4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float4* qr = reinterpret_cast<const float4*>(sq + r * S);
+      const float4* gr = reinterpret_cast<const float4*>(sdo + r * S);
+#pragma unroll 4
+      for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 x = qr[c4], g = gr[c4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const float4 kk = reinterpret_cast<const float4*>(sk + (j0 + jj) * S)[c4];
+          const float4 vv = reinterpret_cast<const float4*>(sv + (j0 + jj) * S)[c4];
+          sv4[jj] = fmaf(x.x, kk.x, fmaf(x.y, kk.y, fmaf(x.z, kk.z, fmaf(x.w, kk.w, sv4[jj]))));
+          dp4[jj] = fmaf(g.x, vv.x, fmaf(g.y, vv.y, fmaf(g.z, vv.z, fmaf(g.w, vv.w, dp4[jj]))));
+        }
+      }
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int j = j0 + jj;
         const bool valid = pos >= 0 && t0 + j <= pos;
-        float s = 0.f, dp = 0.f;
-        if (valid) {
-#pragma unroll 8
-          for (int c = 0; c < D; ++c) {
-            s = fmaf(sq[r * S + c], sk[j * S + c], s);
-            dp = fmaf(sdo[r * S + c], sv[j * S + c], dp);
-          }
-        }
-        const float p = valid ? expf(s * w.scale - s_lse[r]) : 0.f;
+        const float p = valid ? expf(sv4[jj] * w.scale - s_lse[r]) : 0.f;
         sp[r * 8 + j] = p;
-        sds[r * 8 + j] = valid ? p * (dp - s_d[r]) : 0.f;
+        sds[r * 8 + j] = valid ? p * (dp4[jj] - s_d[r]) : 0.f;
       }
     }
     __syncthreads();
@@ -167,22 +174,30 @@ __global__ void __launch_bounds__(kBwThreads) attend_bwd_kernel(BwArgs w) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float ds = sds[rq * 8 + j] * w.scale;
+      const float4* kr = reinterpret_cast<const float4*>(sk + j * S + cq);
 #pragma unroll
-      for (int c = 0; c < kHalfD; ++c) dq[c] = fmaf(ds, sk[j * S + cq + c], dq[c]);
+      for (int c4 = 0; c4 < kHalfD / 4; ++c4) {
+        const float4 kk = kr[c4];
+        dq[4 * c4] = fmaf(ds, kk.x, dq[4 * c4]);
+        dq[4 * c4 + 1] = fmaf(ds, kk.y, dq[4 * c4 + 1]);
+        dq[4 * c4 + 2] = fmaf(ds, kk.z, dq[4 * c4 + 2]);
+        dq[4 * c4 + 3] = fmaf(ds, kk.w, dq[4 * c4 + 3]);
+      }
     }
     // ---- dk, dv of token tid/32, columns 4 (tid%32) .. +4, summed over rows
     {
       const int j = tid >> 5, c0 = (tid & 31) * 4;
       if (c0 < D && t0 + j < T) {
         float4 dk = make_float4(0.f, 0.f, 0.f, 0.f), dv = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
         for (int r = 0; r < kBwRows; ++r) {
           const float ds = sds[r * 8 + j], p = sp[r * 8 + j];
-          const float* qr = sq + r * S + c0;
-          const float* gr = sdo + r * S + c0;
-          dk.x = fmaf(ds, qr[0], dk.x); dk.y = fmaf(ds, qr[1], dk.y);
-          dk.z = fmaf(ds, qr[2], dk.z); dk.w = fmaf(ds, qr[3], dk.w);
-          dv.x = fmaf(p, gr[0], dv.x); dv.y = fmaf(p, gr[1], dv.y);
-          dv.z = fmaf(p, gr[2], dv.z); dv.w = fmaf(p, gr[3], dv.w);
+          const float4 qr = *reinterpret_cast<const float4*>(sq + r * S + c0);
+          const float4 gr = *reinterpret_cast<const float4*>(sdo + r * S + c0);
+          dk.x = fmaf(ds, qr.x, dk.x); dk.y = fmaf(ds, qr.y, dk.y);
+          dk.z = fmaf(ds, qr.z, dk.z); dk.w = fmaf(ds, qr.w, dk.w);
+          dv.x = fmaf(p, gr.x, dv.x); dv.y = fmaf(p, gr.y, dv.y);
+          dv.z = fmaf(p, gr.z, dv.z); dv.w = fmaf(p, gr.w, dv.w);
         }
         dk.x *= w.scale; dk.y *= w.scale; dk.z *= w.scale; dk.w *= w.scale;
         const int64_t off = ((int64_t)h * a.t_cap + t0 + j) * D + c0;
