@@ -129,18 +129,40 @@ __global__ void __launch_bounds__(kBwThreads) attend_bwd_kernel(BwArgs w) {
   const E* kh = static_cast<const E*>(a.k) + (int64_t)h * a.t_cap * D;
   const E* vh = static_cast<const E*>(a.v) + (int64_t)h * a.t_cap * D;
 
+  // K/V of one 8-token group, kPer elements of each per thread; the next
+  // group's loads are issued before the current group's products so that
+  // their latency hides behind them (tokens at or past T, and skipped
+  // entries, read as zero and are never attended)
+  constexpr int kPer = 8 * D / kBwThreads;
+  static_assert(8 * D % kBwThreads == 0, "K/V elements per thread");
+  float kreg[kPer], vreg[kPer];
+  auto fetch = [&](int li) {
+    const int ent = li < n_list ? list[li] : -1;
+    const int64_t g0 = (int64_t)ent * a.group;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int x = tid + i * kBwThreads, j = x / D, c = x % D;
+      const bool in = ent >= 0 && g0 + j < T;
+      kreg[i] = in ? bw_load<E>(kh + (g0 + j) * D + c) : 0.f;
+      vreg[i] = in ? bw_load<E>(vh + (g0 + j) * D + c) : 0.f;
+    }
+  };
+  fetch(0);
   for (int li = 0; li < n_list; ++li) {
-    const int ent = list[li];
-    if (ent < 0) continue;                        // uniform: skipped entry
+    const int ent = list[li];                     // uniform; < 0: skipped entry
     const int64_t t0 = (int64_t)ent * a.group;
-    // the group's 8 tokens of K and V (tokens at or past T are never attended)
-    for (int x = tid; x < 8 * D; x += kBwThreads) {
-      const int j = x / D, c = x % D;
-      const bool in = t0 + j < T;
-      sk[j * S + c] = in ? bw_load<E>(kh + (t0 + j) * D + c) : 0.f;
-      sv[j * S + c] = in ? bw_load<E>(vh + (t0 + j) * D + c) : 0.f;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int x = tid + i * kBwThreads, j = x / D, c = x % D;
+      sk[j * S + c] = kreg[i];
+      sv[j * S + c] = vreg[i];
     }
     __syncthreads();
+    fetch(li + 1);
+    if (ent < 0) {
+      __syncthreads();                            // no products for a skipped entry
+      continue;
+    }
     // ---- p and ds for (row tid/2, tokens 4 (tid%2) .. +4): register tile
     // of 4 dot products of each kind, 16-byte shared loads along d
     {
