@@ -198,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPrThreads, 1)
   bool inv = false;
   if (tid == 0) bars->abort = 0;
   const int n_list = build_group_list(a, b, h, b0, T, list, &n_nondiag, &inv);
-  if (n_list < 0) return;                     // same verdict in both CTAs
+  if (n_list < 0) return;                     // same outcome in both CTAs
   __shared__ int s_inv;
   if (tid == 0) s_inv = 0;
   __syncthreads();

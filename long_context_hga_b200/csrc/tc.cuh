@@ -237,29 +237,6 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
 }
-// Bounded wait with acquire at cluster scope (for arrivals made by the peer).
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort) {
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 0;; ++i) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if ((i & 31) == 31) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        report(HGA_ERR_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
 // Tiled loads issued by either CTA of a pair whose bytes complete on the
 // leader's mbarrier (`leader_bar`, a shared::cluster address); no multicast.
 __device__ __forceinline__ void tma2_load_3d(void* dst, const CUtensorMap* m, int x, int y, int z,
