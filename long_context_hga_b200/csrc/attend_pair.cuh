@@ -128,7 +128,7 @@ __device__ __noinline__ void pair_mma_issuer(PrBars* bars, uint32_t tmem, uint32
     return true;
   };
   auto issue_pv = [&](int j) -> bool {
-    if (!tc::mbar_wait(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
+    if (!tc::mbar_wait_cluster(&bars->p_full[j & 1], (j >> 1) & 1, abort_flag)) return false;
     tc::fence_after_sync();
     const int n = 2 * j + 1, s = n % kPrSlots;
     if (!tc::mbar_wait(&bars->full[s], (n / kPrSlots) & 1, abort_flag)) return false;
@@ -452,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPrThreads, 1)
       tc::fence_before_sync();
       __syncwarp();
       HGA_PR_PH(4);
-      if (lane == 0) tc::mbar_arrive_remote(pfull[x]);
+      if (lane == 0) tc::mbar_arrive_cluster(pfull[x]);
       HGA_PR_PH(5);
       if (lane == 0 && quarter == 0) HGA_PR_TL(rank, 3 + 2 * wg, j);
     }

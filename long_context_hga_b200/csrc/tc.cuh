@@ -229,13 +229,39 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::
                    : "memory");
 }
-// Arrive on an mbarrier of a CTA of the cluster (this CTA's or the peer's),
-// with the default semantics.  The data it announces is in TMEM, ordered by
-// tcgen05.wait::st and tcgen05.fence::before_thread_sync on this side and by
-// tcgen05.fence::after_thread_sync on the waiting side; a cluster-scope
-// release here would cost about a thousand cycles per arrival.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+// Arrive on an mbarrier of a CTA of the cluster (this CTA's or the peer's)
+// with release at cluster scope.  A softmax warp announces P that it stored
+// into its own CTA's TMEM and that the leader CTA's MMA will read: a
+// read-after-write across the pair, so the release (and the waiter's acquire,
+// mbar_wait_cluster) must cover the cluster.  With the default (CTA) scope
+// the leader occasionally read stale P.  The fence costs about a thousand
+// cycles per arrival.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr)
+               : "memory");
+}
+// Bounded wait with acquire at cluster scope (for arrivals made by the peer).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if ((i & 31) == 31) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        report(HGA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
 }
 // Tiled loads issued by either CTA of a pair whose bytes complete on the
 // leader's mbarrier (`leader_bar`, a shared::cluster address); no multicast.
