@@ -698,12 +698,68 @@ def measure_all_configs(args, dev):
             sweep.append({"workload": w.name, "top_chunks": kc, "error": str(exc)[:300]})
     res.append({"workload": gi.SWEEP_32K.name, "budget_sweep": sweep})
     try:
+        res.append(measure_decode(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink))
+    except Exception as exc:
+        res.append({"workload": gi.QWEN3_30B_64K.name, "decode": {"error": str(exc)[:300]}})
+    try:
         res.append(measure_backward(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink))
     except Exception as exc:
         res.append({"workload": gi.QWEN3_30B_64K.name, "backward": {"error": str(exc)[:300]}})
     del flush_w, flush_r
     torch.cuda.empty_cache()
     return res
+
+
+def measure_decode(w, dev, flush_w, flush_r, sink, n_req=8, reps=6):
+    """Generation steps at the 64K context: n_req requests, each with its own
+    K/V cache (the 64K workload's inputs, copied), history committed; one step
+    = hga_decode_step of every request at the 32nd position of its last query
+    block (the block's routing recomputed on its 32 queries), captured as one
+    CUDA graph, cold L2.  Tokens/s = n_req per step.  HBM bytes the method
+    must read per new token: candidate chunk summaries, the kept chunks' group
+    summaries and the attended K/V of every KV head."""
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    pos = w.q0 + 31
+    reqs = []
+    for _ in range(n_req):
+        k, v = inp.k.to(dev), inp.v.to(dev)
+        q = inp.q[:w.qblock].to(dev)                 # queries of the last block so far
+        v16 = torch.empty(v.shape, dtype=torch.float16, device=dev)
+        bufs = hga.allocate(p, w.T, p.qblock, device=dev)
+        hga.commit(p, k, v, 0, w.q0, bufs.chunk_sum, bufs.group_sum, v16)
+        reqs.append((q, k, v, v16, bufs))
+
+    def step():
+        for q, k, v, v16, bufs in reqs:
+            hga.decode_step(p, q, pos, k, v, bufs, v_f16=v16)
+
+    ms = _time_graph(step, reps, 3, flush_w, flush_r, sink)
+    assert hga.check() == 0
+    gc = reqs[0][4].group_cnt.cpu().numpy()
+    b0 = pos - pos % p.qblock
+    n_cand = max(0, (b0 - w.local) // w.chunk - w.sink // w.chunk)
+    kept_chunks = min(w.top_chunks, n_cand) if w.top_chunks > 0 else n_cand
+    routed_groups = float(gc.mean())
+    per_head = (n_cand * w.head_dim * 2                                   # chunk summaries
+                + 8 * kept_chunks * w.head_dim * 2                        # group summaries
+                + (w.sink + routed_groups * w.group + w.local + (pos - b0 + 1))
+                * w.head_dim * 2 * 2)                                     # attended K and V
+    bytes_per_tok = per_head * w.n_kv_heads
+    peaks, kind = load_peaks()
+    achieved = n_req * bytes_per_tok / (ms * 1e-3) / 1e9
+    out = {"workload": w.name, "decode": {
+        "requests": n_req, "position": pos, "ms_per_step": ms,
+        "tokens_per_s": n_req / (ms * 1e-3), "launches_per_step": 4 * n_req,
+        "hbm_bytes_per_token": bytes_per_tok,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "peak_source": f"{kind} copy"},
+        "form": "per request: hga_decode_step (commit, route chunks, route groups, "
+                "attend on the token's block so far); requests not batched into "
+                "one launch"}}
+    return out
 
 
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 flops x 1965 MHz

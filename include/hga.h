@@ -231,6 +231,26 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start,
                        int32_t* group_idx, int32_t* group_cnt, void* o,
                        float* lse, hga_stream_t stream);
 
+/* One generation step of one request (the decode form of the same
+ * method).  The token at position pos has its K/V in the cache and
+ * its query in row pos - b0 of q_block, which holds the queries of its query
+ * block so far (positions b0 .. pos, b0 = pos - pos % qblock; layout of q).
+ * The step commits the token (hga_commit of [b0, pos + 1): summaries of its
+ * group and chunk once closed, and its V in fp16 into v_f16 when v_f16 is not
+ * NULL), routes the block on the queries present and attends: one routing
+ * decision per block, as in prefill (section 6.1 of the page), so the result
+ * equals hga_forward of the segment [b0, pos + 1).  The token's output is row
+ * pos - b0 of o ([n][Hq][d], n = pos - b0 + 1; earlier rows are recomputed
+ * with the block's current routing).  chunk_idx .. group_cnt are sized for one
+ * block; chunk_sum/group_sum hold the committed history.  params.v_f16 must be
+ * 0 (v in dtype); v_f16 must not alias v.  Composed of the calls above; the
+ * pages describe generation only in prose (section 2.2). */
+hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos,
+                           const void* k, const void* v, int64_t t_cap,
+                           void* chunk_sum, void* group_sum, int32_t* chunk_idx,
+                           int32_t* chunk_cnt, int32_t* group_idx, int32_t* group_cnt,
+                           void* v_f16, void* o, float* lse, hga_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Host-memory tier ("Long-Context Fine-Tuning with Limited VRAM", section 2.2
  * tiered KV storage; section 2.1 group summaries in a VRAM cache with misses

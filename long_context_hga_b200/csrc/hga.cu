@@ -645,6 +645,32 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start, int6
   return hga_attend(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
 }
 
+hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos, const void* k,
+                           const void* v, int64_t t_cap, void* chunk_sum, void* group_sum,
+                           int32_t* chunk_idx, int32_t* chunk_cnt, int32_t* group_idx,
+                           int32_t* group_cnt, void* v_f16, void* o, float* lse,
+                           hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if (p->v_f16) return HGA_ERR_INVALID_ARG;       // v is in dtype; v_f16 names the fp16 copy
+  if (pos < 0 || pos >= t_cap) return HGA_ERR_INVALID_ARG;
+  if (v_f16 && v_f16 == v) return HGA_ERR_INVALID_ARG;
+  const int64_t b0 = pos - pos % p->qblock;
+  const int64_t n = pos - b0 + 1;
+  if ((s = hga_commit(p, k, v, t_cap, b0, pos + 1, chunk_sum, group_sum, v_f16, stream)) != HGA_OK)
+    return s;
+  if ((s = hga_route_chunks(p, q_block, b0, n, chunk_sum, t_cap, chunk_idx, chunk_cnt, stream)) !=
+      HGA_OK)
+    return s;
+  if ((s = hga_route_groups(p, q_block, b0, n, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+                            group_cnt, stream)) != HGA_OK)
+    return s;
+  hga_params pa = *p;
+  pa.v_f16 = v_f16 ? 1 : 0;
+  return hga_attend(&pa, q_block, b0, n, k, v_f16 ? v_f16 : v, t_cap, group_idx, group_cnt, o,
+                    lse, stream);
+}
+
 hga_status hga_check(hga_stream_t stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_ok(e);

@@ -28,7 +28,7 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
             "hga_gather_history", "hga_install_group_cache",
             "hga_gather_history_noalloc", "hga_convert_v", "hga_route", "hga_commit",
-            "hga_attend_backward")
+            "hga_attend_backward", "hga_decode_step")
 
 
 class HgaError(RuntimeError):
@@ -105,6 +105,7 @@ def _load() -> ctypes.CDLL:
         "hga_commit": [P, vp, vp, i64, i64, i64, vp, vp, vp, vp],
         "hga_attend_backward": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp,
                                 vp, vp],
+        "hga_decode_step": [P, vp, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -236,6 +237,25 @@ def forward(p: Params, q, q_start: int, k, v, bufs: "Buffers", stream=None):
                         _ptr(bufs.chunk_cnt), _ptr(bufs.group_idx),
                         _ptr(bufs.group_cnt), _ptr(bufs.o), _ptr(bufs.lse),
                         _stream(stream)), "hga_forward")
+
+
+def decode_step(p: Params, q_block, pos: int, k, v, bufs: "Buffers", v_f16=None,
+                stream=None):
+    """One generation step of one request (hga_decode_step): commits the
+    token at `pos`, routes its query block on the queries present in q_block
+    (positions b0 .. pos) and attends; returns the token's output row
+    [Hq][d], a view into bufs.o.  bufs: allocate(p, t_cap, p.qblock), its
+    summaries holding the committed history; v_f16 (optional) receives the
+    token's V in fp16 and is what the attention reads."""
+    b0 = pos - pos % p.qblock
+    n = pos - b0 + 1
+    _ok(LIB.hga_decode_step(ctypes.byref(p.c()), _ptr(q_block[:n]), pos, _ptr(k), _ptr(v),
+                            k.shape[1], _ptr(bufs.chunk_sum), _ptr(bufs.group_sum),
+                            _ptr(bufs.chunk_idx), _ptr(bufs.chunk_cnt), _ptr(bufs.group_idx),
+                            _ptr(bufs.group_cnt), _ptr(v_f16), _ptr(bufs.o[:n]),
+                            None if bufs.lse is None else _ptr(bufs.lse[:n]),
+                            _stream(stream)), "hga_decode_step")
+    return bufs.o[n - 1]
 
 
 @dataclasses.dataclass

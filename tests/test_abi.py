@@ -132,6 +132,14 @@ def test_bad_arguments_rejected_before_launch(hga):
                                  fake, f32, f32, f32, None) == 1
     assert L.hga_attend_backward(pp, None, 0, 0, None, None, 1024, None, None, None, None,
                                  None, None, None, None, None) == 0
+    # decode step: position outside the cache, fp16 copy aliasing v, params
+    # that already say fp16 V
+    assert L.hga_decode_step(pp, fake, 1024, fake, fake, 1024, fake, fake, fake, fake, fake,
+                             fake, None, fake, None, None) == 1
+    assert L.hga_decode_step(pp, fake, 70, fake, fake, 1024, fake, fake, fake, fake, fake,
+                             fake, fake, fake, None, None) == 1
+    assert L.hga_decode_step(ctypes.byref(p16), fake, 70, fake, fake, 1024, fake, fake, fake,
+                             fake, fake, fake, None, fake, None, None) == 1
     # empty work is a no-op, not an error
     assert L.hga_build_summaries(pp, None, 1024, 64, 64, None, None, None) == 0
     assert L.hga_route_chunks(pp, None, 0, 0, None, 1024, None, None, None) == 0
