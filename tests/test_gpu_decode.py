@@ -63,3 +63,34 @@ def test_decode_steps_match_oracle_and_prefill(v16):
         for h in range(w.n_kv_heads):
             if res.group_margin[(0, h)] > 1e-4 and res.chunk_margin[(0, h)] > 1e-4:
                 assert list(gi_np[h, 0, :gc_np[h, 0]]) == res.group_idx[(0, h)], (pos, h)
+
+
+def test_lockstep_requests_as_heads_equal_separate_steps():
+    """Requests decoding at the same position can share one call: request r's
+    KV heads become heads r*Hkv .. of one cache and its query heads r*Hq ..;
+    every (block, KV head) unit is independent, so the outputs equal the
+    per-request steps bit for bit."""
+    from long_context_hga_b200 import hga
+    dev = torch.device("cuda:0")
+    ws = [gi.QWEN3_30B_64K.with_(T=2112, q0=2048, seed=s, n_needles=2) for s in (0, 1)]
+    p = hga.Params.from_workload(ws[0])
+    pos = 2048 + 40
+    outs, qs, ks, vs = [], [], [], []
+    for w in ws:
+        inp = gi.make_inputs(w)
+        q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+        bufs = hga.allocate(p, w.T, p.qblock, device=dev)
+        hga.commit(p, k, v, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+        outs.append(hga.decode_step(p, q, pos, k, v, bufs).clone())
+        qs.append(q)
+        ks.append(k)
+        vs.append(v)
+    pb = dataclasses.replace(p, n_q_heads=2 * p.n_q_heads, n_kv_heads=2 * p.n_kv_heads)
+    kb, vb = torch.cat(ks, 0), torch.cat(vs, 0)
+    qb = torch.cat(qs, 1).contiguous()
+    bb = hga.allocate(pb, ws[0].T, p.qblock, device=dev)
+    hga.commit(pb, kb, vb, 0, ws[0].q0, bb.chunk_sum, bb.group_sum)
+    row = hga.decode_step(pb, qb, pos, kb, vb, bb)
+    assert hga.check() == 0
+    assert torch.equal(row[:p.n_q_heads], outs[0])
+    assert torch.equal(row[p.n_q_heads:], outs[1])
