@@ -712,12 +712,14 @@ def measure_all_configs(args, dev):
 
 def measure_decode(w, dev, flush_w, flush_r, sink, n_req=8, reps=6):
     """Generation steps at the 64K context: n_req requests, each with its own
-    K/V cache (the 64K workload's inputs, copied), history committed; one step
-    = hga_decode_step of every request at the 32nd position of its last query
-    block (the block's routing recomputed on its 32 queries), captured as one
-    CUDA graph, cold L2.  Tokens/s = n_req per step.  HBM bytes the method
-    must read per new token: candidate chunk summaries, the kept chunks' group
-    summaries and the attended K/V of every KV head."""
+    K/V cache (copies of the 64K workload's inputs), history committed; one
+    step decodes the token at the 32nd position of every request's last query
+    block (the block's routing recomputed on its 32 queries).  Timed two ways,
+    each as one CUDA graph with a cold L2: one hga_decode_step per request,
+    and the requests in lockstep as the heads of a single call.  Tokens/s =
+    n_req per step.  HBM bytes the method must read per new token: candidate
+    chunk summaries, the kept chunks' group summaries and the attended K/V of
+    every KV head."""
     from long_context_hga_b200 import hga
     p = hga.Params.from_workload(w)
     inp = gi.make_inputs(w)
