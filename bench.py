@@ -663,6 +663,109 @@ def measure_tiered(w, dev, flush_w, flush_r, sink, steps=5):
             "pcie_bytes_per_step": (int(tier.bytes.item()) - b0) / steps}
 
 
+def _filesystem_of(path):
+    """(mount point, type, device) of the filesystem holding path."""
+    best = ("?", "?", "?")
+    try:
+        real = os.path.realpath(path)
+        for line in open("/proc/mounts"):
+            dev_, mnt, typ = line.split()[:3]
+            if (real == mnt or real.startswith(mnt.rstrip("/") + "/")) and \
+                    len(mnt) >= len(best[0].replace("?", "")):
+                best = (mnt, typ, dev_)
+    except OSError:
+        pass
+    return {"mount": best[0], "type": best[1], "device": best[2]}
+
+
+def measure_store(w, dev, cold_steps=3, warm_steps=5, page_tokens=64, io_threads=16):
+    """Tiered step of the 128K workload with the history's K/V in a file
+    (pages of 64 tokens of one KV head, K then V) read through a page cache
+    in pinned RAM bounded to the pages one step needs (found by a first step
+    with room for the whole history); group summaries as in the RAM tier.
+    Cold steps start with an empty cache and read with O_DIRECT when the
+    filesystem allows it (so the OS page cache does not serve them); warm
+    steps find every page cached.  Wall-clock per step (the host waits for
+    the routing and fills the cache inside the step)."""
+    import shutil
+    import tempfile
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    q = inp.q.to(dev)
+    full = hga.allocate(p, w.T, w.Tq, device=dev)
+    k_seg = inp.k.to(dev)
+    hga.build_summaries(p, k_seg, 0, w.q0, full.chunk_sum, full.group_sum)
+    del k_seg
+    tier = hga.make_host_tier(p, None, None, full.group_sum.cpu().pin_memory(), t_hist=w.q0)
+    k_dev = torch.zeros(w.n_kv_heads, w.T, w.head_dim, dtype=torch.bfloat16, device=dev)
+    v_dev = torch.zeros_like(k_dev)
+    k_dev[:, w.q0:] = inp.k[:, w.q0:].to(dev)
+    v_dev[:, w.q0:] = inp.v[:, w.q0:].to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    bufs.chunk_sum.copy_(full.chunk_sum)
+    tmp = tempfile.mkdtemp(prefix="hga_store_")
+    path = os.path.join(tmp, "kv.bin")
+    try:
+        hist_pages = w.n_kv_heads * (-(-w.q0 // page_tokens))
+        direct = True
+        try:
+            store = hga.KVStore(p, path, w.T, page_tokens, hist_pages, direct=True)
+        except hga.HgaError:
+            direct = False
+            store = hga.KVStore(p, path, w.T, page_tokens, hist_pages, direct=False)
+        t0 = time.perf_counter()
+        store.append(inp.k[:, :w.q0].contiguous(), inp.v[:, :w.q0].contiguous())
+        with open(path, "rb+") as f:
+            os.fsync(f.fileno())
+        write_s = time.perf_counter() - t0
+
+        def one():
+            torch.cuda.synchronize()
+            t = time.perf_counter()
+            st = hga.store_step(p, q, w.q0, tier, store, k_dev, v_dev, bufs, io_threads)
+            torch.cuda.synchronize()
+            st["ms"] = (time.perf_counter() - t) * 1e3
+            return st
+
+        store.reset_cache()
+        cache_pages = one()["pages_needed"]          # probe: the bound for the cache
+        cold = []
+        for _ in range(cold_steps):
+            store.reset_cache(cache_pages)
+            cold.append(one())
+        warm = [one() for _ in range(warm_steps)]
+        assert hga.check() == 0
+        # the step's output against the all-HBM path (same inputs, HBM-resident history)
+        k_all, v_all = inp.k.to(dev), inp.v.to(dev)
+        hga.forward(p, q, w.q0, k_all, v_all, full)
+        same = bool(torch.equal(full.o, bufs.o))
+        del k_all, v_all
+        store.close()
+    finally:
+        shutil.rmtree(tmp, ignore_errors=True)
+    med = lambda xs: float(np.median(xs))
+    c0 = cold[-1]
+    cold_ms = med([c["ms"] for c in cold])
+    cold_prep = med([c["prepare_s"] for c in cold])
+    return {"workload": w.name, "store": {
+        "file": {"bytes": hist_pages * store.page_bytes, "page_bytes": store.page_bytes,
+                 "o_direct_reads": direct, "filesystem": _filesystem_of(tmp),
+                 "append_and_fsync_s": write_s},
+        "cache_pages": cache_pages, "history_pages": hist_pages,
+        "io_threads": io_threads,
+        "pages_needed_per_step": c0["pages_needed"],
+        "cold": {"ms_per_step": cold_ms, "query_tokens_per_s": w.Tq / (cold_ms * 1e-3),
+                 "bytes_read": c0["bytes_read"], "prepare_ms": cold_prep * 1e3,
+                 "read_GBps": c0["bytes_read"] / max(cold_prep, 1e-9) / 1e9},
+        "warm": {"ms_per_step": med([c["ms"] for c in warm]),
+                 "query_tokens_per_s": w.Tq / (med([c["ms"] for c in warm]) * 1e-3),
+                 "hits": warm[-1]["hits"], "misses": warm[-1]["misses"],
+                 "prepare_ms": med([c["prepare_s"] for c in warm]) * 1e3},
+        "output_equals_all_hbm_step": same,
+        "timing": "wall clock per store_step with a device synchronise on both sides"}}
+
+
 def measure_all_configs(args, dev):
     """Every other workload, briefly (the headline line times the 64K one)."""
     flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -678,6 +781,10 @@ def measure_all_configs(args, dev):
         res.append(measure_tiered(gi.TIERED_128K, dev, flush_w, flush_r, sink))
     except Exception as exc:
         res.append({"workload": gi.TIERED_128K.name, "error": str(exc)[:300]})
+    try:
+        res.append(measure_store(gi.TIERED_128K, dev))
+    except Exception as exc:
+        res.append({"workload": gi.TIERED_128K.name, "store": {"error": str(exc)[:300]}})
     # budget sweep at 32K: sparsity vs throughput vs max error against dense
     sweep = []
     dense_o = None

@@ -75,7 +75,9 @@ typedef enum {
   HGA_ERR_UNSUPPORTED = 2,   /* legal but not built: dtype, head_dim, sizes     */
   HGA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed            */
   HGA_ERR_DEVICE_CHECK = 4,  /* a kernel found an out-of-range index (hga_check)*/
-  HGA_ERR_TIMEOUT = 5        /* a bounded device wait gave up (hga_check)       */
+  HGA_ERR_TIMEOUT = 5,       /* a bounded device wait gave up (hga_check)       */
+  HGA_ERR_IO = 6,            /* a file open, read or write failed (K/V store)   */
+  HGA_ERR_CAPACITY = 7       /* the store's page cache cannot hold one step     */
 } hga_status;
 
 typedef enum { HGA_BF16 = 0, HGA_FP32 = 1 } hga_dtype;
@@ -325,6 +327,118 @@ hga_status hga_gather_history_noalloc(const hga_params* p, int64_t q_start, int6
                                       const int32_t* group_cnt, const void* k_host,
                                       const void* v_host, void* k_dev, void* v_dev,
                                       unsigned long long* bytes, hga_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * File-backed K/V store ("Long-Context Fine-Tuning with Limited VRAM",
+ * section 2.2: besides RAM-backed history the method has a filesystem store
+ * in which RAM is a bounded page cache over disk, suited to NVMe; section 6.2
+ * notes it was not benchmarked there).  The history's exact K/V lives in one
+ * file; a step's routed, sink and local-window history groups are read into a
+ * bounded page cache in pinned host memory, from which a kernel gathers them
+ * into the device mirrors (as hga_gather_history does from whole-history
+ * RAM).  Group summaries keep using the RAM tier above.
+ *
+ * File layout: pages of page_tokens tokens of one KV head; page (h, n) holds
+ * K then V, each [page_tokens][head_dim] in the store's dtype, at byte offset
+ * (h * n_pages + n) * page_bytes, page_bytes = 2 * page_tokens * head_dim *
+ * elem_size, n_pages = ceil(t_cap / page_tokens).  Tokens never appended read
+ * as zeros.  Cache slot i occupies cache[i * page_bytes ..) with the page's
+ * file image.  page_table[h * n_pages + n] = the slot holding page (h, n), or
+ * -1; it is written only by the store.
+ *
+ * Step:  route chunks -> hga_fetch_group_summaries -> hga_route_groups ->
+ *        copy group_idx/group_cnt to the host, synchronise ->
+ *        hga_store_prepare (misses read from the file, least recently used
+ *        pages evicted) -> hga_gather_store -> hga_attend.
+ * Results equal the all-HBM path's exactly.
+ *
+ * Threading: a store is not thread-safe; calls on one store are serial.
+ * hga_store_prepare and hga_store_append rewrite cache slots and page_table:
+ * the caller makes sure no hga_gather_store of this store is still running
+ * (e.g. the synchronisation before hga_store_prepare covers the previous
+ * step's gather when both run on one stream). */
+typedef struct hga_kv_store hga_kv_store;
+
+typedef struct hga_store_stats {
+  int64_t pages_needed;   /* distinct (KV head, page) the step reads           */
+  int64_t hits;           /* of those, already in the cache                     */
+  int64_t misses;         /* read from the file                                 */
+  int64_t evictions;      /* cached pages dropped to make room                  */
+  int64_t bytes_read;     /* file bytes read                                    */
+} hga_store_stats;
+
+#define HGA_STORE_CREATE 1   /* create or truncate the file to its full size   */
+#define HGA_STORE_DIRECT 2   /* read with O_DIRECT (bypasses the OS page cache; */
+                             /* page_bytes and the cache must be 4096-aligned)  */
+
+/* Opens the store file `path` for the layout of p (n_kv_heads, head_dim,
+ * dtype) and context capacity t_cap.  page_tokens: a positive multiple of
+ * p->group.  Without HGA_STORE_CREATE the file must exist and have the full
+ * size; its length (tokens appended) starts at 0 and is set by
+ * hga_store_append or hga_store_set_length.  *out receives the handle
+ * (NULL on error).  Errors: HGA_ERR_INVALID_ARG, HGA_ERR_IO (open/truncate
+ * failed, or O_DIRECT refused by the filesystem). */
+hga_status hga_store_open(const char* path, const hga_params* p, int64_t t_cap,
+                          int64_t page_tokens, int32_t flags, hga_kv_store** out);
+
+/* Closes the file and frees the handle (the file stays).  NULL is a no-op. */
+hga_status hga_store_close(hga_kv_store* s);
+
+/* Gives the store its page cache: cache_pages slots of page_bytes at `cache`
+ * and page_table [n_kv_heads][n_pages] int32, both caller-owned host memory
+ * (pinned when a kernel reads them) that must outlive the store or the next
+ * attach.  Every slot starts empty; page_table is filled with -1. */
+hga_status hga_store_attach_cache(hga_kv_store* s, void* cache, int64_t cache_pages,
+                                  int32_t* page_table);
+
+/* Appends n tokens of K and V at the current length: k, v are host arrays
+ * [n_kv_heads][n][head_dim] in the store's dtype.  Cached pages that the
+ * tokens touch are updated too.  HGA_ERR_INVALID_ARG when length + n > t_cap. */
+hga_status hga_store_append(hga_kv_store* s, const void* k, const void* v, int64_t n);
+
+/* Declares the first `length` tokens of an existing file valid (reopening a
+ * store written earlier).  0 <= length <= t_cap. */
+hga_status hga_store_set_length(hga_kv_store* s, int64_t length);
+
+/* Tokens appended (or declared), -1 for NULL. */
+int64_t hga_store_length(const hga_kv_store* s);
+
+/* Bytes of one page (K and V), -1 for NULL. */
+int64_t hga_store_page_bytes(const hga_kv_store* s);
+
+/* Pages per KV head, -1 for NULL. */
+int64_t hga_store_pages_per_head(const hga_kv_store* s);
+
+/* Reads tokens [t_begin, t_end) of K and V straight from the file into host
+ * arrays [n_kv_heads][t_end - t_begin][head_dim] (the cache is not used). */
+hga_status hga_store_read(hga_kv_store* s, int64_t t_begin, int64_t t_end, void* k, void* v);
+
+/* Makes every page the step's history groups fall in resident: for each
+ * (block, KV head) the sink groups, the routed groups group_idx/group_cnt
+ * (HOST copies, layouts as hga_route_groups writes them for s's t_cap) and
+ * the local-window groups that lie below t_hist.  Resident pages are marked
+ * used; missing ones take free slots, else the least recently used slots
+ * that this step does not need, and are read from the file by io_threads
+ * threads (>= 1).  t_hist: a multiple of p->group, <= q_start and <= the
+ * store's length.  *stats (when not NULL) receives this call's counts.
+ * Errors: HGA_ERR_INVALID_ARG; HGA_ERR_CAPACITY when the step needs more
+ * pages than the cache has (pages loaded so far stay valid); HGA_ERR_IO when
+ * a read fails (that page stays absent). */
+hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_start,
+                             int64_t n_q, int64_t t_hist, const int32_t* group_idx,
+                             const int32_t* group_cnt, int32_t io_threads,
+                             hga_store_stats* stats);
+
+/* hga_gather_history with the store's page cache as the source: copies the
+ * same history groups from their cache slots into k_dev/v_dev (device
+ * [n_kv_heads][t_cap][head_dim]), each (KV head, group) once per step (gen,
+ * step as in hga_gather_history).  group_idx/group_cnt are the DEVICE
+ * arrays.  A group whose page is not resident sets HGA_ERR_DEVICE_CHECK
+ * (hga_check) and is skipped: call hga_store_prepare first. */
+hga_status hga_gather_store(const hga_params* p, const hga_kv_store* s, int64_t q_start,
+                            int64_t n_q, int64_t t_hist, const int32_t* group_idx,
+                            const int32_t* group_cnt, void* k_dev, void* v_dev, uint32_t* gen,
+                            uint32_t step, unsigned long long* bytes, hga_stream_t stream);
 
 /* Slots per (KV head, block) of chunk_idx (which = 0) or group_idx
  * (which = 1) for a context capacity t_cap; -1 on invalid parameters. */

@@ -33,6 +33,8 @@ def _nvcc() -> str:
 def sources() -> list:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) +
                   glob.glob(os.path.join(CSRC, "*.cuh")) +
+                  glob.glob(os.path.join(CSRC, "*.cpp")) +
+                  glob.glob(os.path.join(CSRC, "*.h")) +
                   glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
@@ -47,7 +49,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not is_stale():
         return LIB
     cmd = [_nvcc(), *NVCC_FLAGS, *extra, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "hga.cu"), "-o", LIB + ".tmp"]
+           os.path.join(CSRC, "hga.cu"), os.path.join(CSRC, "kv_store.cpp"),
+           "-o", LIB + ".tmp"]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)

@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "hga.h"
+#include "kv_store.h"
 #include "common.cuh"
 #include "summaries.cuh"
 #include "route.cuh"
@@ -689,6 +690,8 @@ const char* hga_status_string(hga_status s) {
     case HGA_ERR_CUDA: return "HGA_ERR_CUDA";
     case HGA_ERR_DEVICE_CHECK: return "HGA_ERR_DEVICE_CHECK";
     case HGA_ERR_TIMEOUT: return "HGA_ERR_TIMEOUT";
+    case HGA_ERR_IO: return "HGA_ERR_IO";
+    case HGA_ERR_CAPACITY: return "HGA_ERR_CAPACITY";
   }
   return "HGA_ERR_UNKNOWN";
 }
@@ -810,6 +813,39 @@ hga_status hga_gather_history(const hga_params* p, int64_t q_start, int64_t n_q,
                       group_cnt, reinterpret_cast<const T*>(k_host),
                       reinterpret_cast<const T*>(v_host), reinterpret_cast<T*>(k_dev),
                       reinterpret_cast<T*>(v_dev), gen, step, bytes);
+  };
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? go(__nv_bfloat16{}, std::integral_constant<int, 128>{})
+                              : go(__nv_bfloat16{}, std::integral_constant<int, 64>{});
+  return p->head_dim == 128 ? go(float{}, std::integral_constant<int, 128>{})
+                            : go(float{}, std::integral_constant<int, 64>{});
+}
+
+hga_status hga_gather_store(const hga_params* p, const hga_kv_store* store, int64_t q_start,
+                            int64_t n_q, int64_t t_hist, const int32_t* group_idx,
+                            const int32_t* group_cnt, void* k_dev, void* v_dev, uint32_t* gen,
+                            uint32_t step, unsigned long long* bytes, hga_stream_t stream) {
+  if (!p || !store) return HGA_ERR_INVALID_ARG;
+  hga::TierArgs a;
+  hga_status s = tier_args(p, q_start, n_q, store->t_cap, t_hist, &a);
+  if (s != HGA_OK) return s;
+  if (p->n_kv_heads != store->Hkv || p->head_dim != store->d || p->dtype != store->dtype)
+    return HGA_ERR_INVALID_ARG;
+  if (t_hist > store->length) return HGA_ERR_INVALID_ARG;
+  if (n_q == 0) return HGA_OK;
+  if (!store->cache || !store->page_table || !group_idx || !group_cnt || !k_dev || !v_dev ||
+      !gen || step == 0)
+    return HGA_ERR_INVALID_ARG;
+  hga::StoreArgs sa{store->cache, store->page_table, store->n_pages, store->page_tokens,
+                    store->cache_pages, store->half_bytes};
+  dim3 grid(a.n_blocks, a.Hkv);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto go = [&](auto tag, auto dim) {
+    using T = decltype(tag);
+    constexpr int D = decltype(dim)::value;
+    return launch_pdl(hga::gather_store_kernel<D, T>, grid, dim3(256), 0, st, a, sa, group_idx,
+                      group_cnt, reinterpret_cast<T*>(k_dev), reinterpret_cast<T*>(v_dev), gen,
+                      step, bytes);
   };
   if (p->dtype == HGA_BF16)
     return p->head_dim == 128 ? go(__nv_bfloat16{}, std::integral_constant<int, 128>{})

@@ -130,6 +130,65 @@ __global__ void __launch_bounds__(256) gather_history_kernel(
   if (lane == 0 && bytes && copied) atomicAdd(bytes, copied);
 }
 
+// gather_history_kernel with a file-backed store's page cache as the source
+// (section 2.2: RAM as a bounded page cache over the disk store).  The host
+// made every page the step needs resident (hga_store_prepare); page_table
+// maps (KV head, page) to its cache slot, whose image is the page's K half
+// then its V half, [page_tokens][D] each.  A group whose page is absent sets
+// the device check and is skipped.
+struct StoreArgs {
+  const char* cache;             // host page cache (pinned, read over PCIe)
+  const int32_t* page_table;     // [Hkv][n_pages]
+  int64_t n_pages, page_tokens, cache_pages, half_bytes;
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(256) gather_store_kernel(
+    TierArgs a, StoreArgs sa, const int32_t* __restrict__ group_idx,
+    const int32_t* __restrict__ group_cnt, T* __restrict__ k_dev, T* __restrict__ v_dev,
+    uint32_t* __restrict__ gen, uint32_t step, unsigned long long* __restrict__ bytes) {
+  griddep_wait();
+  const int b = blockIdx.x, h = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
+  const int g = a.group;
+  const int64_t sink_end = min((int64_t)a.sink, b0);
+  const int n_s = (int)(sink_end / g);
+  int n_r = group_cnt[(int64_t)h * a.n_blocks + b];
+  if (n_r < 0 || n_r > a.cap_g) n_r = 0;
+  const int32_t* routed = group_idx + ((int64_t)h * a.n_blocks + b) * a.cap_g;
+  const int64_t loc_lo = max(sink_end, b0 - a.local);
+  const int n_l = (int)((b0 - loc_lo) / g);
+  unsigned long long copied = 0;
+  for (int i = warp; i < n_s + n_r + n_l; i += 8) {
+    int64_t j;
+    if (i < n_s) j = i;
+    else if (i < n_s + n_r) j = routed[i - n_s];
+    else j = loc_lo / g + (i - n_s - n_r);
+    if (j < 0 || (j + 1) * g > a.t_hist) continue;            // resident, or invalid
+    const int64_t t = j * g;
+    const int64_t pg = t / sa.page_tokens;
+    const int32_t slot = pg < sa.n_pages ? sa.page_table[(int64_t)h * sa.n_pages + pg] : -1;
+    if (slot < 0 || slot >= sa.cache_pages) {
+      if (lane == 0) report(HGA_ERR_DEVICE_CHECK);
+      continue;
+    }
+    uint32_t prev = 0;
+    if (lane == 0) prev = atomicExch(&gen[(int64_t)h * a.n_groups_cap + j], step);
+    prev = __shfl_sync(0xffffffffu, prev, 0);
+    if (prev == step) continue;                               // already fetched this step
+    const char* page = sa.cache + (int64_t)slot * 2 * sa.half_bytes +
+                       (t - pg * sa.page_tokens) * D * (int64_t)sizeof(T);
+    const int64_t off = ((int64_t)h * a.t_cap + t) * D;
+    warp_copy(page, reinterpret_cast<char*>(k_dev + off), g * D * (int)sizeof(T), lane);
+    warp_copy(page + sa.half_bytes, reinterpret_cast<char*>(v_dev + off),
+              g * D * (int)sizeof(T), lane);
+    copied += 2ull * g * D * sizeof(T);
+  }
+  griddep_launch();
+  if (lane == 0 && bytes && copied) atomicAdd(bytes, copied);
+}
+
 // Each claimed slot takes its claim (the largest group that missed on it).
 template <int D, typename T>
 __global__ void __launch_bounds__(256) install_group_cache_kernel(

@@ -10,6 +10,7 @@ from __future__ import annotations
 import ctypes
 import dataclasses
 import os
+import time
 from typing import Optional
 
 import torch
@@ -19,6 +20,8 @@ LIB_PATH = os.path.join(_PKG, "libhga.so")
 
 HGA_OK, HGA_ERR_INVALID_ARG, HGA_ERR_UNSUPPORTED = 0, 1, 2
 HGA_ERR_CUDA, HGA_ERR_DEVICE_CHECK, HGA_ERR_TIMEOUT = 3, 4, 5
+HGA_ERR_IO, HGA_ERR_CAPACITY = 6, 7
+HGA_STORE_CREATE, HGA_STORE_DIRECT = 1, 2
 HGA_BF16, HGA_FP32 = 0, 1
 
 EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
@@ -28,7 +31,10 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_set_kernel_variant", "hga_selftest_exp2", "hga_fetch_group_summaries",
             "hga_gather_history", "hga_install_group_cache",
             "hga_gather_history_noalloc", "hga_convert_v", "hga_route", "hga_commit",
-            "hga_attend_backward", "hga_decode_step")
+            "hga_attend_backward", "hga_decode_step", "hga_store_open", "hga_store_close",
+            "hga_store_attach_cache", "hga_store_append", "hga_store_set_length",
+            "hga_store_length", "hga_store_page_bytes", "hga_store_pages_per_head",
+            "hga_store_read", "hga_store_prepare", "hga_gather_store")
 
 
 class HgaError(RuntimeError):
@@ -355,12 +361,14 @@ class HostTier:
                            self.stats.data_ptr())
 
 
-def make_host_tier(p: Params, k_host: torch.Tensor, v_host: torch.Tensor,
+def make_host_tier(p: Params, k_host: Optional[torch.Tensor], v_host: Optional[torch.Tensor],
                    gsum_host: torch.Tensor, t_hist: int, cache_fraction: float = 0.25,
                    device="cuda") -> HostTier:
-    """k_host/v_host/gsum_host: pinned CPU tensors in the all-HBM layouts."""
+    """k_host/v_host/gsum_host: pinned CPU tensors in the all-HBM layouts.
+    k_host/v_host may be None when the history K/V lives in a KVStore (the
+    tier then serves the group summaries only)."""
     for t in (k_host, v_host, gsum_host):
-        if not t.is_pinned():
+        if t is not None and not t.is_pinned():
             raise ValueError("host tier tensors must be pinned")
     Hkv, n_groups = gsum_host.shape[0], gsum_host.shape[1]
     cap = max(1, int(-(-cache_fraction * Hkv * n_groups // Hkv)))
@@ -433,3 +441,177 @@ def tiered_step(p: Params, q, q_start: int, tier: HostTier, k_dev, v_dev, bufs: 
     main.wait_stream(side)
     attend(p, q, q_start, k_dev, v_dev, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
     install_group_cache(p, t_cap, tier)
+
+
+# ---------------------------------------------------------------- file-backed store
+
+class CStoreStats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "pages_needed", "hits", "misses", "evictions", "bytes_read")]
+
+
+def _sig_store():
+    P = ctypes.POINTER(CParams)
+    vp, i64, i32, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32
+    sig = {
+        "hga_store_open": [ctypes.c_char_p, P, i64, i64, i32, ctypes.POINTER(vp)],
+        "hga_store_close": [vp],
+        "hga_store_attach_cache": [vp, vp, i64, vp],
+        "hga_store_append": [vp, vp, vp, i64],
+        "hga_store_set_length": [vp, i64],
+        "hga_store_read": [vp, i64, i64, vp, vp],
+        "hga_store_prepare": [vp, P, i64, i64, i64, vp, vp, i32, ctypes.POINTER(CStoreStats)],
+        "hga_gather_store": [P, vp, i64, i64, i64, vp, vp, vp, vp, vp, u32, vp, vp],
+    }
+    for name, args in sig.items():
+        fn = getattr(LIB, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    for name in ("hga_store_length", "hga_store_page_bytes", "hga_store_pages_per_head"):
+        getattr(LIB, name).argtypes = [vp]
+        getattr(LIB, name).restype = ctypes.c_int64
+
+
+_sig_store()
+
+
+def _aligned_bytes(n: int, align: int, pin: bool) -> torch.Tensor:
+    raw = torch.empty(n + align, dtype=torch.uint8, pin_memory=pin)
+    off = (-raw.data_ptr()) % align
+    return raw[off:off + n]
+
+
+class KVStore:
+    """History K/V in one file, read through a bounded page cache in host
+    memory (pinned when a kernel gathers from it).  A page is page_tokens
+    tokens of one KV head, K then V; the page table [Hkv][n_pages] maps a
+    page to its cache slot (-1 absent).  Wraps the hga_store_* calls."""
+
+    def __init__(self, p: Params, path: str, t_cap: int, page_tokens: int, cache_pages: int,
+                 create: bool = True, direct: bool = False, pin: bool = True):
+        self.p, self.path, self.t_cap = p, path, t_cap
+        h = ctypes.c_void_p()
+        flags = (HGA_STORE_CREATE if create else 0) | (HGA_STORE_DIRECT if direct else 0)
+        _ok(LIB.hga_store_open(path.encode(), ctypes.byref(p.c()), t_cap, page_tokens, flags,
+                               ctypes.byref(h)), "hga_store_open")
+        self.handle = h
+        self.page_tokens = page_tokens
+        self.page_bytes = int(LIB.hga_store_page_bytes(h))
+        self.n_pages = int(LIB.hga_store_pages_per_head(h))
+        self.cache_pages = cache_pages
+        self.cache = _aligned_bytes(cache_pages * self.page_bytes, 4096, pin)
+        self.page_table = _aligned_bytes(p.n_kv_heads * self.n_pages * 4, 64, pin).view(
+            torch.int32).view(p.n_kv_heads, self.n_pages)
+        _ok(LIB.hga_store_attach_cache(h, _ptr(self.cache), cache_pages, _ptr(self.page_table)),
+            "hga_store_attach_cache")
+        self._host_idx = None
+
+    @property
+    def length(self) -> int:
+        return int(LIB.hga_store_length(self.handle))
+
+    def set_length(self, n: int):
+        _ok(LIB.hga_store_set_length(self.handle, n), "hga_store_set_length")
+
+    def append(self, k: torch.Tensor, v: torch.Tensor):
+        """k, v: CPU [Hkv][n][d] in the store's dtype."""
+        k, v = k.contiguous(), v.contiguous()
+        if k.device.type != "cpu" or v.device.type != "cpu" or k.shape != v.shape:
+            raise ValueError("append takes two CPU tensors of one shape [Hkv][n][d]")
+        _ok(LIB.hga_store_append(self.handle, _ptr(k), _ptr(v), k.shape[1]), "hga_store_append")
+
+    def read(self, t_begin: int, t_end: int):
+        """Tokens [t_begin, t_end) from the file: CPU K, V [Hkv][n][d]."""
+        shape = (self.p.n_kv_heads, t_end - t_begin, self.p.head_dim)
+        k = torch.empty(shape, dtype=self.p.torch_dtype)
+        v = torch.empty(shape, dtype=self.p.torch_dtype)
+        _ok(LIB.hga_store_read(self.handle, t_begin, t_end, _ptr(k), _ptr(v)), "hga_store_read")
+        return k, v
+
+    def prepare(self, p: Params, q_start: int, n_q: int, t_hist: int, group_idx_host,
+                group_cnt_host, io_threads: int = 8) -> dict:
+        st = CStoreStats()
+        code = LIB.hga_store_prepare(self.handle, ctypes.byref(p.c()), q_start, n_q, t_hist,
+                                     _ptr(group_idx_host), _ptr(group_cnt_host), io_threads,
+                                     ctypes.byref(st))
+        stats = {n: getattr(st, n) for n, _ in CStoreStats._fields_}
+        _ok(code, "hga_store_prepare")
+        return stats
+
+    def reset_cache(self, cache_pages: Optional[int] = None):
+        """Drops every cached page (the slots and the page table restart
+        empty); cache_pages, at most the allocated count, bounds the cache
+        from now on."""
+        n = self.cache_pages if cache_pages is None else cache_pages
+        if not 0 < n <= self.cache.numel() // self.page_bytes:
+            raise ValueError("cache_pages exceeds the allocated cache")
+        _ok(LIB.hga_store_attach_cache(self.handle, _ptr(self.cache), n,
+                                       _ptr(self.page_table)), "hga_store_attach_cache")
+        self.cache_pages = n
+
+    def host_index_buffers(self, bufs: "Buffers"):
+        """Pinned host copies' storage for a step's group_idx / group_cnt."""
+        if (self._host_idx is None or self._host_idx[0].shape != bufs.group_idx.shape
+                or self._host_idx[1].shape != bufs.group_cnt.shape):
+            self._host_idx = (torch.empty(bufs.group_idx.shape, dtype=torch.int32,
+                                          pin_memory=True),
+                              torch.empty(bufs.group_cnt.shape, dtype=torch.int32,
+                                          pin_memory=True))
+        return self._host_idx
+
+    def close(self):
+        if self.handle:
+            code = LIB.hga_store_close(self.handle)
+            self.handle = None
+            _ok(code, "hga_store_close")
+
+    def __del__(self):
+        try:
+            if getattr(self, "handle", None):
+                LIB.hga_store_close(self.handle)
+                self.handle = None
+        except Exception:
+            pass
+
+
+def gather_store(p: Params, store: KVStore, q_start: int, n_q: int, t_hist: int, group_idx,
+                 group_cnt, k_dev, v_dev, gen, step: int, nbytes=None, stream=None):
+    _ok(LIB.hga_gather_store(ctypes.byref(p.c()), store.handle, q_start, n_q, t_hist,
+                             _ptr(group_idx), _ptr(group_cnt), _ptr(k_dev), _ptr(v_dev),
+                             _ptr(gen), ctypes.c_uint32(step), _ptr(nbytes), _stream(stream)),
+        "hga_gather_store")
+
+
+def store_step(p: Params, q, q_start: int, tier: HostTier, store: KVStore, k_dev, v_dev,
+               bufs: "Buffers", io_threads: int = 8) -> dict:
+    """One query segment with the history K/V in a file-backed store: segment
+    summaries, chunk routing, group-summary fetch (HBM cache / pinned RAM),
+    group routing, the routed indices to the host, the store's page cache
+    filled from the file, history gathered from the cache, attention, cache
+    install.  Everything runs on the current stream; the host waits once,
+    for the indices.  Returns the store's counts for the step, with the
+    host's wait for the routing (host_wait_s) and the time the cache took to
+    fill (prepare_s)."""
+    main = torch.cuda.current_stream()
+    n_q, t_cap = q.shape[0], k_dev.shape[1]
+    build_summaries(p, k_dev, q_start, q_start + n_q, bufs.chunk_sum, bufs.group_sum)
+    route_chunks(p, q, q_start, bufs.chunk_sum, t_cap, bufs.chunk_idx, bufs.chunk_cnt)
+    fetch_group_summaries(p, q_start, n_q, t_cap, tier, bufs.chunk_idx, bufs.chunk_cnt,
+                          bufs.group_sum)
+    route_groups(p, q, q_start, bufs.group_sum, t_cap, bufs.chunk_idx, bufs.chunk_cnt,
+                 bufs.group_idx, bufs.group_cnt)
+    gi_h, gc_h = store.host_index_buffers(bufs)
+    gi_h.copy_(bufs.group_idx, non_blocking=True)
+    gc_h.copy_(bufs.group_cnt, non_blocking=True)
+    t0 = time.perf_counter()
+    main.synchronize()                  # also ends the previous step's gather
+    t1 = time.perf_counter()
+    stats = store.prepare(p, q_start, n_q, tier.t_hist, gi_h, gc_h, io_threads)
+    stats["host_wait_s"] = t1 - t0
+    stats["prepare_s"] = time.perf_counter() - t1
+    tier.step += 1
+    gather_store(p, store, q_start, n_q, tier.t_hist, bufs.group_idx, bufs.group_cnt, k_dev,
+                 v_dev, tier.gen, tier.step, tier.bytes)
+    attend(p, q, q_start, k_dev, v_dev, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse)
+    install_group_cache(p, t_cap, tier)
+    return stats

@@ -34,7 +34,8 @@ def test_exports_every_declared_symbol(hga):
 def test_status_strings(hga):
     for code, name in [(0, "HGA_OK"), (1, "HGA_ERR_INVALID_ARG"),
                        (2, "HGA_ERR_UNSUPPORTED"), (3, "HGA_ERR_CUDA"),
-                       (4, "HGA_ERR_DEVICE_CHECK"), (5, "HGA_ERR_TIMEOUT")]:
+                       (4, "HGA_ERR_DEVICE_CHECK"), (5, "HGA_ERR_TIMEOUT"),
+                       (6, "HGA_ERR_IO"), (7, "HGA_ERR_CAPACITY")]:
         assert hga.status_string(code) == name
 
 
