@@ -33,7 +33,11 @@ Readings where the pages are silent (each is also listed in the design notes):
     asc); k <= 0 means all; the group budget is global over the groups of the
     chosen chunks;
   * margin = k-th selected score minus best unselected score (+inf when all
-    candidates are taken), in scaled units.
+    candidates are taken), in scaled units;
+  * strictly causal routing variant (section 6.1 names it and leaves its
+    design to future work): block b is routed on the queries of the block
+    before it (positions b0 - qblock .. b0 - qblock + n - 1 for a block of n
+    rows), so no position's output depends on a later input.
 
 Parity pins (none of the pages' worked numbers exist; see tests/): dense
 equivalence at full budget against torch's CPU scaled_dot_product_attention,
@@ -176,8 +180,33 @@ def select_top(cands: list, scores: np.ndarray, k: int):
     return chosen, margin
 
 
-def route_chunks_unit(q, q0, T, csum_h, p: Params, b: int, h: int):
-    rows, b0, _ = block_rows(q, q0, T, p, b, h)
+def causal_route_queries(q_before: np.ndarray, q: np.ndarray) -> np.ndarray:
+    """Routing queries of the strictly causal variant, indexed like q: row i
+    is the query at position q0 + i - qblock.  q_before [qblock][Hq][d] holds
+    the queries of the qblock positions before q0 (any values when q0 = 0:
+    the first block of a sequence has no candidates)."""
+    return np.concatenate([q_before, q], axis=0)[:q.shape[0]]
+
+
+def routing_rows(q, q0, T, p: Params, b: int, h: int, q_route=None):
+    """Rows that score the summaries for block b, as an [n * G][d] matrix,
+    plus b0 and b1.  Standard HGA (section 2.1; section 6.1 notes that one
+    routing decision serves every position of the block): the block's own
+    queries.  Strictly causal variant (section 6.1 leaves its design open;
+    reading: the block is routed on the queries of the block before it, as
+    many rows as the block has): rows b*qblock .. b*qblock + n - 1 of
+    q_route (see causal_route_queries), i.e. positions b0 - qblock ..
+    b1 - qblock - 1, all before the block's first token."""
+    rows, b0, b1 = block_rows(q, q0, T, p, b, h)
+    if q_route is None:
+        return rows, b0, b1
+    i0 = b * p.qblock
+    r = q_route[i0:i0 + (b1 - b0), h * p.G:(h + 1) * p.G, :]
+    return r.reshape(-1, q.shape[-1]), b0, b1
+
+
+def route_chunks_unit(q, q0, T, csum_h, p: Params, b: int, h: int, q_route=None):
+    rows, b0, _ = routing_rows(q, q0, T, p, b, h, q_route)
     cands = chunk_candidates(b0, p)
     if not cands:
         return [], math.inf
@@ -186,8 +215,8 @@ def route_chunks_unit(q, q0, T, csum_h, p: Params, b: int, h: int):
 
 
 def route_groups_unit(q, q0, T, gsum_h, chunks: list, p: Params, b: int,
-                      h: int):
-    rows, _, _ = block_rows(q, q0, T, p, b, h)
+                      h: int, q_route=None):
+    rows, _, _ = routing_rows(q, q0, T, p, b, h, q_route)
     per = p.chunk // p.group
     cands = [c * per + i for c in chunks for i in range(per)]
     if not cands:
@@ -258,12 +287,14 @@ def n_blocks(q0: int, T: int, p: Params) -> int:
 
 
 def hga_forward(q, k, v, q0: int, p: Params, units=None, csum=None,
-                gsum=None, with_attention: bool = True) -> Result:
+                gsum=None, with_attention: bool = True, q_route=None) -> Result:
     """Run the four steps for the query segment [q0, T).
 
     q [Tq][Hq][d], k and v [Hkv][T][d], float64 holding the exact storage
     values.  `units` restricts the work to a list of (block, kv_head) pairs
-    (default: all).  Summaries cover [0, T) unless given."""
+    (default: all).  Summaries cover [0, T) unless given.  q_route (from
+    causal_route_queries) selects the strictly causal routing variant;
+    attention always uses q."""
     T = k.shape[1]
     if csum is None or gsum is None:
         csum, gsum = build_summaries(k, p, 0, T)
@@ -272,8 +303,8 @@ def hga_forward(q, k, v, q0: int, p: Params, units=None, csum=None,
                  for b in range(n_blocks(q0, T, p))]
     res = Result()
     for (b, h) in units:
-        ch, cm = route_chunks_unit(q, q0, T, csum[h], p, b, h)
-        gr, gm = route_groups_unit(q, q0, T, gsum[h], ch, p, b, h)
+        ch, cm = route_chunks_unit(q, q0, T, csum[h], p, b, h, q_route)
+        gr, gm = route_groups_unit(q, q0, T, gsum[h], ch, p, b, h, q_route)
         res.chunk_idx[(b, h)] = ch
         res.chunk_margin[(b, h)] = cm
         res.group_idx[(b, h)] = gr

@@ -89,9 +89,9 @@ def _round_truncate(x):                  # chops instead of rounding to even
     return np.ldexp(np.trunc(np.ldexp(m, 8)), e - 8)
 
 
-def _group_per_chunk_quota(q, q0, T, gsum_h, chunks, p, b, h):
+def _group_per_chunk_quota(q, q0, T, gsum_h, chunks, p, b, h, q_route=None):
     # best groups chosen per chunk instead of over all chosen chunks
-    rows, _, _ = ho.block_rows(q, q0, T, p, b, h)
+    rows, _, _ = ho.routing_rows(q, q0, T, p, b, h, q_route)
     per = p.chunk // p.group
     out = []
     for c in chunks:
