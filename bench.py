@@ -812,6 +812,11 @@ def measure_all_configs(args, dev):
         res.append(measure_backward(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink))
     except Exception as exc:
         res.append({"workload": gi.QWEN3_30B_64K.name, "backward": {"error": str(exc)[:300]}})
+    try:
+        res.append(measure_causal(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink))
+    except Exception as exc:
+        res.append({"workload": gi.QWEN3_30B_64K.name,
+                    "causal_routing": {"error": str(exc)[:300]}})
     del flush_w, flush_r
     torch.cuda.empty_cache()
     return res
@@ -942,6 +947,45 @@ def measure_backward(w, dev, flush_w, flush_r, sink, reps=6):
                      "frac": tf / FP32_ALU_PEAK_TFLOPS,
                      "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
         "kernel": "fp32 CUDA cores, one CTA per 128-row slice, 16-byte atomics for dK/dV"}}
+
+
+def measure_causal(w, dev, flush_w, flush_r, sink, reps=6):
+    """Strictly causal routing variant (each block routed on the block before
+    it) against the block-shared routing, same inputs: device time of
+    hga_forward_causal and hga_forward (segment summaries, both routings,
+    attention; bf16 V) with a cold L2, eager launches between CUDA events."""
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    q_ext = torch.cat([gi.make_q_before(w), inp.q]).to(dev)
+    q = q_ext[w.qblock:]
+    k, v = inp.k.to(dev), inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush_w.zero_()
+            torch.sum(flush_r, 0, out=sink)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        assert hga.check() == 0
+        return float(np.median(ts))
+
+    ms_shared = timed(lambda: hga.forward(p, q, w.q0, k, v, bufs))
+    o_shared = bufs.o.clone()
+    ms_causal = timed(lambda: hga.forward_causal(p, q_ext, w.q0, k, v, bufs))
+    return {"workload": w.name, "causal_routing": {
+        "ms": ms_causal, "query_tokens_per_s": w.Tq / (ms_causal * 1e-3),
+        "block_shared_ms": ms_shared, "ratio_to_block_shared": ms_causal / ms_shared,
+        "max_abs_diff_vs_block_shared": float((bufs.o.float() - o_shared.float()).abs().max()),
+        "timing": "eager launches between CUDA events, cold L2, median of 6"}}
 
 
 def run_reference(args, world, rank):

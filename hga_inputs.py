@@ -151,6 +151,23 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Inputs:
     return Inputs(w, qt, kt, vt, needles)
 
 
+def make_q_before(w: Workload, seed: Optional[int] = None) -> torch.Tensor:
+    """The qblock queries at positions q0 - qblock .. q0 - 1, [qblock][Hq][d]
+    in the storage dtype: standard normal rows rotated at their positions,
+    drawn from their own stream (seed + 2).  All zero when q0 < qblock (no
+    earlier positions exist).  They feed the strictly causal routing
+    variant, which routes the segment's first block on them."""
+    seed = w.seed if seed is None else seed
+    B, Hq, d = w.qblock, w.n_q_heads, w.head_dim
+    if w.q0 < B:
+        return _round(np.zeros((B, Hq, d)), w.dtype)
+    rng = np.random.Generator(np.random.PCG64(seed + 2))
+    q = rng.standard_normal((B, Hq, d), dtype=np.float32)
+    cos_q, sin_q = _rope_tables(np.arange(w.q0 - B, w.q0), d, w.rope_theta)
+    q64 = _apply_rope(q.astype(np.float64).transpose(1, 0, 2), cos_q, sin_q)
+    return _round(q64.transpose(1, 0, 2), w.dtype)
+
+
 def _plant_needles(w: Workload, q64: np.ndarray, k_out: np.ndarray,
                    seed: int) -> list:
     """Replace the keys of n_needles groups per KV head in k_out (in place)."""

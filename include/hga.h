@@ -253,6 +253,27 @@ hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos
                            int32_t* chunk_cnt, int32_t* group_idx, int32_t* group_cnt,
                            void* v_f16, void* o, float* lse, hga_stream_t stream);
 
+/* Strictly causal routing variant ("Long-Context Fine-Tuning with Limited
+ * VRAM", section 6.1: sharing one routing decision across a block lets an
+ * earlier token learn about later ones; a strictly causal variant is named
+ * and its design left to future work).  This library's reading: block b is
+ * routed on the queries of the block before it, as many rows as b has
+ * (positions b0 - qblock .. b0 - qblock + n_b - 1), which all precede the
+ * block's first token, so no output depends on a later input.  Same cost as
+ * hga_forward.
+ *   q_ext: [qblock + n_q][n_q_heads][head_dim]; rows 0..qblock-1 are the
+ *          queries at positions q_start - qblock .. q_start - 1 (any finite
+ *          values when q_start == 0: the first block of a sequence has no
+ *          candidates), rows qblock.. the segment's queries.
+ * Other arguments, layouts and errors as hga_forward.  The result equals
+ * hga_route_chunks + hga_route_groups called with q = q_ext (routing) and
+ * hga_attend with q = q_ext + qblock rows, after the segment's summaries. */
+hga_status hga_forward_causal(const hga_params* p, const void* q_ext, int64_t q_start,
+                              int64_t n_q, const void* k, const void* v, int64_t t_cap,
+                              void* chunk_sum, void* group_sum, int32_t* chunk_idx,
+                              int32_t* chunk_cnt, int32_t* group_idx, int32_t* group_cnt, void* o,
+                              float* lse, hga_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * Host-memory tier ("Long-Context Fine-Tuning with Limited VRAM", section 2.2
  * tiered KV storage; section 2.1 group summaries in a VRAM cache with misses

@@ -646,6 +646,33 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start, int6
   return hga_attend(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
 }
 
+hga_status hga_forward_causal(const hga_params* p, const void* q_ext, int64_t q_start,
+                              int64_t n_q, const void* k, const void* v, int64_t t_cap,
+                              void* chunk_sum, void* group_sum, int32_t* chunk_idx,
+                              int32_t* chunk_cnt, int32_t* group_idx, int32_t* group_cnt, void* o,
+                              float* lse, hga_stream_t stream) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
+  if (n_q > 0 && !q_ext) return HGA_ERR_INVALID_ARG;
+  // routing reads rows [b*qblock, ..) of q_ext = the block before block b;
+  // attention reads the segment's own queries, qblock rows further on
+  const size_t elem = p->dtype == HGA_BF16 ? 2 : 4;
+  const void* q = q_ext ? static_cast<const char*>(q_ext) +
+                              (size_t)p->qblock * p->n_q_heads * p->head_dim * elem
+                        : nullptr;
+  if ((s = hga_build_summaries(p, k, t_cap, q_start, q_start + n_q, chunk_sum, group_sum,
+                               stream)) != HGA_OK)
+    return s;
+  if ((s = hga_route_chunks(p, q_ext, q_start, n_q, chunk_sum, t_cap, chunk_idx, chunk_cnt,
+                            stream)) != HGA_OK)
+    return s;
+  if ((s = hga_route_groups(p, q_ext, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt,
+                            group_idx, group_cnt, stream)) != HGA_OK)
+    return s;
+  return hga_attend(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
+}
+
 hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos, const void* k,
                            const void* v, int64_t t_cap, void* chunk_sum, void* group_sum,
                            int32_t* chunk_idx, int32_t* chunk_cnt, int32_t* group_idx,

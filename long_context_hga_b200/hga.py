@@ -34,7 +34,7 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_attend_backward", "hga_decode_step", "hga_store_open", "hga_store_close",
             "hga_store_attach_cache", "hga_store_append", "hga_store_set_length",
             "hga_store_length", "hga_store_page_bytes", "hga_store_pages_per_head",
-            "hga_store_read", "hga_store_prepare", "hga_gather_store")
+            "hga_store_read", "hga_store_prepare", "hga_gather_store", "hga_forward_causal")
 
 
 class HgaError(RuntimeError):
@@ -112,6 +112,8 @@ def _load() -> ctypes.CDLL:
         "hga_attend_backward": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp,
                                 vp, vp],
         "hga_decode_step": [P, vp, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "hga_forward_causal": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp, vp,
+                               vp, vp, vp],
     }
     for name, args in sig.items():
         fn = getattr(lib, name)
@@ -243,6 +245,21 @@ def forward(p: Params, q, q_start: int, k, v, bufs: "Buffers", stream=None):
                         _ptr(bufs.chunk_cnt), _ptr(bufs.group_idx),
                         _ptr(bufs.group_cnt), _ptr(bufs.o), _ptr(bufs.lse),
                         _stream(stream)), "hga_forward")
+
+
+def forward_causal(p: Params, q_ext, q_start: int, k, v, bufs: "Buffers", stream=None):
+    """Strictly causal routing variant: q_ext = the qblock queries before
+    q_start followed by the segment's queries; block b is routed on the block
+    before it, attention uses the segment's own queries."""
+    n_q = q_ext.shape[0] - p.qblock
+    if n_q < 0:
+        raise HgaError(HGA_ERR_INVALID_ARG, "forward_causal: q_ext shorter than one block")
+    _ok(LIB.hga_forward_causal(ctypes.byref(p.c()), _ptr(q_ext), q_start, n_q,
+                               _ptr(k), _ptr(v), k.shape[1], _ptr(bufs.chunk_sum),
+                               _ptr(bufs.group_sum), _ptr(bufs.chunk_idx),
+                               _ptr(bufs.chunk_cnt), _ptr(bufs.group_idx),
+                               _ptr(bufs.group_cnt), _ptr(bufs.o), _ptr(bufs.lse),
+                               _stream(stream)), "hga_forward_causal")
 
 
 def decode_step(p: Params, q_block, pos: int, k, v, bufs: "Buffers", v_f16=None,

@@ -44,6 +44,27 @@ class GpuResult:
     lse: np.ndarray
 
 
+def run_gpu_causal(w: gi.Workload, inp: gi.Inputs, q_before) -> GpuResult:
+    """Strictly causal routing variant: history summaries [0, q0) first, then
+    hga_forward_causal on q_before followed by the segment's queries."""
+    from long_context_hga_b200 import hga
+    p = hga.Params.from_workload(w)
+    dev = torch.device("cuda:0")
+    q_ext = torch.cat([q_before, inp.q]).to(dev)
+    k, v = inp.k.to(dev), inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    if w.q0 > 0:
+        hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+    hga.forward_causal(p, q_ext, w.q0, k, v, bufs)
+    st = hga.check()
+    assert st == 0, f"device status {hga.status_string(st)}"
+    f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+    return GpuResult(f(bufs.chunk_sum), f(bufs.group_sum),
+                     bufs.chunk_idx.cpu().numpy(), bufs.chunk_cnt.cpu().numpy(),
+                     bufs.group_idx.cpu().numpy(), bufs.group_cnt.cpu().numpy(),
+                     f(bufs.o), bufs.lse.cpu().numpy().astype(np.float64))
+
+
 def run_gpu(w: gi.Workload, inp: gi.Inputs, t_cap: Optional[int] = None,
             split_history: bool = True, v_f16: bool = False) -> GpuResult:
     """History summaries [0, q0) are built first (the committed history), then
@@ -124,7 +145,9 @@ def _valid_choice(chosen, cands, scores, k, band=NEAR_TIE) -> bool:
 
 
 def compare(w: gi.Workload, inp: gi.Inputs, gpu: GpuResult, units=None,
-            check_summaries: bool = True) -> Report:
+            check_summaries: bool = True, q_route=None) -> Report:
+    """q_route (float64, from oracle causal_route_queries) compares against
+    the strictly causal routing variant instead of the block-shared one."""
     p = oracle_params(w)
     q = gi.to_f64(inp.q)
     k = gi.to_f64(inp.k)
@@ -146,8 +169,8 @@ def compare(w: gi.Workload, inp: gi.Inputs, gpu: GpuResult, units=None,
     causal_total = 0
     for (b, h) in units:
         rep.units += 1
-        rows, b0, b1 = ho.block_rows(q, q0, T, p, b, h)
-        ch_ref, ch_margin = ho.route_chunks_unit(q, q0, T, csum[h], p, b, h)
+        rows, b0, b1 = ho.routing_rows(q, q0, T, p, b, h, q_route)
+        ch_ref, ch_margin = ho.route_chunks_unit(q, q0, T, csum[h], p, b, h, q_route)
         ch_gpu = [int(x) for x in gpu.chunk_idx[h, b, :gpu.chunk_cnt[h, b]]]
         cap = gpu.chunk_idx.shape[2]
         pad_ok = (gpu.chunk_idx[h, b, gpu.chunk_cnt[h, b]:] == -1).all()
@@ -163,7 +186,8 @@ def compare(w: gi.Workload, inp: gi.Inputs, gpu: GpuResult, units=None,
             rep.chunk_mismatch += 1
         if not chunk_same:
             continue
-        gr_ref, gr_margin = ho.route_groups_unit(q, q0, T, gsum[h], ch_ref, p, b, h)
+        gr_ref, gr_margin = ho.route_groups_unit(q, q0, T, gsum[h], ch_ref, p, b, h,
+                                                 q_route)
         gr_gpu = [int(x) for x in gpu.group_idx[h, b, :gpu.group_cnt[h, b]]]
         gpad_ok = (gpu.group_idx[h, b, gpu.group_cnt[h, b]:] == -1).all()
         group_same = gr_gpu == gr_ref

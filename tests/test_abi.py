@@ -141,6 +141,13 @@ def test_bad_arguments_rejected_before_launch(hga):
                              fake, fake, fake, None, None) == 1
     assert L.hga_decode_step(ctypes.byref(p16), fake, 70, fake, fake, 1024, fake, fake, fake,
                              fake, fake, fake, None, fake, None, None) == 1
+    # causal-routing forward: no query buffer, a segment off the block grid
+    assert L.hga_forward_causal(pp, None, 64, 64, fake, fake, 1024, fake, fake, fake, fake,
+                                fake, fake, fake, None, None) == 1
+    assert L.hga_forward_causal(pp, fake, 32, 64, fake, fake, 1024, fake, fake, fake, fake,
+                                fake, fake, fake, None, None) == 1
+    assert L.hga_forward_causal(pp, None, 64, 0, None, None, 1024, None, None, None, None,
+                                None, None, None, None, None) == 0
     # empty work is a no-op, not an error
     assert L.hga_build_summaries(pp, None, 1024, 64, 64, None, None, None) == 0
     assert L.hga_route_chunks(pp, None, 0, 0, None, 1024, None, None, None) == 0

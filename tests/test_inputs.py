@@ -40,3 +40,21 @@ def test_needles_are_candidates():
         c = j * w.group // w.chunk
         assert c * w.chunk >= w.sink and (c + 1) * w.chunk <= b0 - w.local
         assert 0 <= b < w.Tq // w.qblock
+
+
+def test_q_before_shape_determinism_and_rotation():
+    """The queries before a segment: [qblock][Hq][d] in the storage dtype,
+    the same draw every call, zero when no earlier position exists, and
+    rotated at their own positions (RoPE keeps each pair's norm)."""
+    w = gi.QWEN3_30B_64K.with_(T=8168, q0=6144)
+    a, b = gi.make_q_before(w), gi.make_q_before(w)
+    assert a.shape == (w.qblock, w.n_q_heads, w.head_dim) and a.dtype == torch.bfloat16
+    assert torch.equal(a, b)
+    assert not gi.make_q_before(gi.TINY_FP32).any()
+    rng = np.random.Generator(np.random.PCG64(w.seed + 2))
+    raw = rng.standard_normal((w.qblock, w.n_q_heads, w.head_dim), dtype=np.float32)
+    half = w.head_dim // 2
+    norm = lambda x: np.sqrt(x[..., :half] ** 2 + x[..., half:] ** 2)
+    got = a.float().numpy().astype(np.float64)
+    assert np.allclose(norm(got), norm(raw.astype(np.float64)), rtol=2e-2, atol=2e-2)
+    assert not np.allclose(got, raw, atol=1e-2)          # rotated, not the raw draw
