@@ -158,15 +158,22 @@ hga_status hga_store_attach_cache(hga_kv_store* s, void* cache, int64_t cache_pa
   // 16-byte rows for the gather kernel's vector copies; 4096 for O_DIRECT reads
   if (reinterpret_cast<uintptr_t>(cache) % (s->direct ? 4096 : 16)) return HGA_ERR_INVALID_ARG;
   const int64_t n_global = s->Hkv * s->n_pages;
+  try {                                         // no C++ exception crosses the C ABI
+    s->slot_page.assign((size_t)cache_pages, -1);
+    s->prev.assign((size_t)cache_pages, -1);
+    s->next.assign((size_t)cache_pages, -1);
+    s->slot_step.assign((size_t)cache_pages, 0);
+    s->page_step.assign((size_t)n_global, 0);
+    s->free_slots.resize((size_t)cache_pages);
+  } catch (...) {
+    s->cache = nullptr;
+    s->page_table = nullptr;
+    s->cache_pages = 0;
+    return HGA_ERR_INVALID_ARG;
+  }
   s->cache = static_cast<char*>(cache);
   s->cache_pages = cache_pages;
   s->page_table = page_table;
-  s->slot_page.assign((size_t)cache_pages, -1);
-  s->prev.assign((size_t)cache_pages, -1);
-  s->next.assign((size_t)cache_pages, -1);
-  s->slot_step.assign((size_t)cache_pages, 0);
-  s->page_step.assign((size_t)n_global, 0);
-  s->free_slots.resize((size_t)cache_pages);
   for (int64_t i = 0; i < cache_pages; ++i) s->free_slots[(size_t)i] = (int32_t)(cache_pages - 1 - i);
   s->lru_head = s->lru_tail = -1;
   s->step = 0;
@@ -265,6 +272,13 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
   const uint32_t step = s->step;
   hga_store_stats c{};
   std::vector<int64_t> missing;
+  std::vector<int32_t> slots;
+  std::vector<char> ok;
+  try {                                         // reserve up front: no throw below
+    missing.reserve((size_t)std::min<int64_t>(s->cache_pages, s->Hkv * s->n_pages));
+  } catch (...) {
+    return HGA_ERR_INVALID_ARG;
+  }
   for (int64_t h = 0; h < s->Hkv; ++h) {
     for (int64_t b = 0; b < n_blocks; ++b) {
       const int64_t b0 = q_start + b * p->qblock;
@@ -291,9 +305,9 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
           s->slot_step[(size_t)slot] = step;
           lru_unlink(s, slot);
           lru_push_front(s, slot);
-        } else {
+        } else if (missing.size() < missing.capacity()) {
           missing.push_back(gp);
-        }
+        }   // else: more misses than slots, so pages_needed > cache_pages below
       }
     }
   }
@@ -304,7 +318,13 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
 
   // slots for the missing pages: free ones first, then the least recently
   // used pages this step does not need (they sit at the tail of the list)
-  std::vector<int32_t> slots(missing.size());
+  try {
+    slots.resize(missing.size());
+    ok.assign(missing.size(), 0);
+  } catch (...) {
+    if (stats) *stats = c;
+    return HGA_ERR_INVALID_ARG;
+  }
   for (size_t i = 0; i < missing.size(); ++i) {
     int32_t slot;
     if (!s->free_slots.empty()) {
@@ -332,7 +352,6 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
   }
 
   // reads, several in flight
-  std::vector<char> ok(missing.size(), 0);
   auto worker = [&](std::atomic<size_t>* next) {
     for (size_t i; (i = next->fetch_add(1)) < missing.size();) {
       char* dst = s->cache + (int64_t)slots[i] * s->page_bytes;
@@ -345,8 +364,11 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
     worker(&next);
   } else {
     std::vector<std::thread> pool;
-    pool.reserve(n_thr - 1);
-    for (size_t t = 1; t < n_thr; ++t) pool.emplace_back(worker, &next);
+    try {                                       // fewer threads if the system refuses some
+      pool.reserve(n_thr - 1);
+      for (size_t t = 1; t < n_thr; ++t) pool.emplace_back(worker, &next);
+    } catch (...) {
+    }
     worker(&next);
     for (auto& th : pool) th.join();
   }
