@@ -452,9 +452,10 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
 
 /* hga_gather_history with the store's page cache as the source: copies the
  * same history groups from their cache slots into k_dev/v_dev (device
- * [n_kv_heads][t_cap][head_dim]), each (KV head, group) once per step (gen,
- * step as in hga_gather_history).  group_idx/group_cnt are the DEVICE
- * arrays.  A group whose page is not resident sets HGA_ERR_DEVICE_CHECK
+ * [n_kv_heads][t_cap][head_dim], t_cap = the store's, as given to
+ * hga_store_open), each (KV head, group) once per step (gen, step as in
+ * hga_gather_history).  group_idx/group_cnt are the DEVICE arrays, laid out
+ * for the store's t_cap.  A group whose page is not resident sets HGA_ERR_DEVICE_CHECK
  * (hga_check) and is skipped: call hga_store_prepare first. */
 hga_status hga_gather_store(const hga_params* p, const hga_kv_store* s, int64_t q_start,
                             int64_t n_q, int64_t t_hist, const int32_t* group_idx,

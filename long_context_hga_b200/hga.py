@@ -593,6 +593,10 @@ class KVStore:
 
 def gather_store(p: Params, store: KVStore, q_start: int, n_q: int, t_hist: int, group_idx,
                  group_cnt, k_dev, v_dev, gen, step: int, nbytes=None, stream=None):
+    """k_dev/v_dev: device [Hkv][store.t_cap][d]; group_idx/group_cnt laid out
+    for store.t_cap."""
+    if k_dev.shape[1] != store.t_cap or v_dev.shape[1] != store.t_cap:
+        raise HgaError(HGA_ERR_INVALID_ARG, "gather_store: k_dev/v_dev must span the store's t_cap")
     _ok(LIB.hga_gather_store(ctypes.byref(p.c()), store.handle, q_start, n_q, t_hist,
                              _ptr(group_idx), _ptr(group_cnt), _ptr(k_dev), _ptr(v_dev),
                              _ptr(gen), ctypes.c_uint32(step), _ptr(nbytes), _stream(stream)),
@@ -611,6 +615,8 @@ def store_step(p: Params, q, q_start: int, tier: HostTier, store: KVStore, k_dev
     fill (prepare_s)."""
     main = torch.cuda.current_stream()
     n_q, t_cap = q.shape[0], k_dev.shape[1]
+    if t_cap != store.t_cap or v_dev.shape[1] != store.t_cap:
+        raise HgaError(HGA_ERR_INVALID_ARG, "store_step: k_dev/v_dev must span the store's t_cap")
     build_summaries(p, k_dev, q_start, q_start + n_q, bufs.chunk_sum, bufs.group_sum)
     route_chunks(p, q, q_start, bufs.chunk_sum, t_cap, bufs.chunk_idx, bufs.chunk_cnt)
     fetch_group_summaries(p, q_start, n_q, t_cap, tier, bufs.chunk_idx, bufs.chunk_cnt,
