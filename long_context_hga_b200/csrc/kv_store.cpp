@@ -17,6 +17,7 @@
 #include <fcntl.h>
 #include <string.h>
 #include <sys/stat.h>
+#include <sys/uio.h>
 #include <unistd.h>
 
 #include <algorithm>
@@ -25,6 +26,8 @@
 #include <thread>
 
 namespace {
+
+constexpr int64_t kMaxRunPages = 256;           // iovecs per vectored read (<= IOV_MAX)
 
 bool pread_full(int fd, char* dst, int64_t bytes, int64_t off) {
   while (bytes > 0) {
@@ -40,6 +43,33 @@ bool pread_full(int fd, char* dst, int64_t bytes, int64_t off) {
     dst += r;
     off += r;
     bytes -= r;
+  }
+  return true;
+}
+
+// Reads one contiguous file range into scattered buffers (one run of
+// adjacent pages into their cache slots); zero-fills past the end of file.
+bool preadv_full(int fd, struct iovec* iov, int n, int64_t off) {
+  int i = 0;
+  while (i < n) {
+    ssize_t r = ::preadv(fd, iov + i, n - i, (off_t)off);
+    if (r < 0) {
+      if (errno == EINTR) continue;
+      return false;
+    }
+    if (r == 0) {
+      for (; i < n; ++i) memset(iov[i].iov_base, 0, iov[i].iov_len);
+      return true;
+    }
+    off += r;
+    while (i < n && (size_t)r >= iov[i].iov_len) {
+      r -= (ssize_t)iov[i].iov_len;
+      ++i;
+    }
+    if (i < n && r > 0) {
+      iov[i].iov_base = static_cast<char*>(iov[i].iov_base) + r;
+      iov[i].iov_len -= (size_t)r;
+    }
   }
   return true;
 }
@@ -274,6 +304,7 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
   std::vector<int64_t> missing;
   std::vector<int32_t> slots;
   std::vector<char> ok;
+  std::vector<std::pair<size_t, size_t>> runs;   // (first index in missing, pages)
   try {                                         // reserve up front: no throw below
     missing.reserve((size_t)std::min<int64_t>(s->cache_pages, s->Hkv * s->n_pages));
   } catch (...) {
@@ -315,6 +346,7 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
     if (stats) *stats = c;
     return HGA_ERR_CAPACITY;
   }
+  std::sort(missing.begin(), missing.end());    // file order, for runs of adjacent pages
 
   // slots for the missing pages: free ones first, then the least recently
   // used pages this step does not need (they sit at the tail of the list)
@@ -351,15 +383,41 @@ hga_status hga_store_prepare(hga_kv_store* s, const hga_params* p, int64_t q_sta
     slots[i] = slot;
   }
 
-  // reads, several in flight
+  // reads, several in flight: runs of pages adjacent in the file (missing is
+  // sorted) go into one vectored read of up to 1 MiB, each page to its slot
+  const size_t max_run = (size_t)std::max<int64_t>(
+      1, std::min<int64_t>(kMaxRunPages, (1 << 20) / s->page_bytes));
+  try {
+    for (size_t i = 0; i < missing.size();) {
+      size_t n = 1;
+      while (i + n < missing.size() && n < max_run && missing[i + n] == missing[i] + (int64_t)n) ++n;
+      runs.emplace_back(i, n);
+      i += n;
+    }
+  } catch (...) {
+    runs.clear();
+    for (size_t i = 0; i < missing.size(); ++i) {
+      s->slot_page[(size_t)slots[i]] = -1;
+      lru_unlink(s, slots[i]);
+      s->free_slots.push_back(slots[i]);
+    }
+    if (stats) *stats = c;
+    return HGA_ERR_INVALID_ARG;
+  }
   auto worker = [&](std::atomic<size_t>* next) {
-    for (size_t i; (i = next->fetch_add(1)) < missing.size();) {
-      char* dst = s->cache + (int64_t)slots[i] * s->page_bytes;
-      ok[i] = pread_full(s->fd_read, dst, s->page_bytes, missing[i] * s->page_bytes) ? 1 : 0;
+    struct iovec iov[kMaxRunPages];
+    for (size_t r; (r = next->fetch_add(1)) < runs.size();) {
+      const size_t i0 = runs[r].first, n = runs[r].second;
+      for (size_t j = 0; j < n; ++j) {
+        iov[j].iov_base = s->cache + (int64_t)slots[i0 + j] * s->page_bytes;
+        iov[j].iov_len = (size_t)s->page_bytes;
+      }
+      const char good = preadv_full(s->fd_read, iov, (int)n, missing[i0] * s->page_bytes);
+      for (size_t j = 0; j < n; ++j) ok[i0 + j] = good;
     }
   };
   std::atomic<size_t> next{0};
-  const size_t n_thr = std::min<size_t>((size_t)io_threads, missing.size());
+  const size_t n_thr = std::min<size_t>((size_t)io_threads, runs.size());
   if (n_thr <= 1) {
     worker(&next);
   } else {
