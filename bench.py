@@ -470,6 +470,10 @@ def run_hga(args, world, rank, local):
         value = n_tok / (ms * 1e-3)
         kernels = {name: round(float(per_kernel[:, j].mean()) * 1e3, 2)
                    for j, name in enumerate(names)}
+        # information, not a target: planted needle groups the routing kept for
+        # the block each was planted for (read after the timed region)
+        g_idx, g_cnt = bufs.group_idx.cpu().numpy(), bufs.group_cnt.cpu().numpy()
+        found = sum(int(j in g_idx[h, b, :g_cnt[h, b]]) for (h, j, b) in inp.needles)
         out = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -497,6 +501,10 @@ def run_hga(args, world, rank, local):
                             (float(sum(per_kernel[:, col[n]] for n in col if n.startswith("route")).mean())
                              * 1e-3) / 1e12,
             "density": counts["density"],
+            "step_ms_percentiles": {k_: float(np.percentile(step_ms, q_))
+                                    for k_, q_ in (("p10", 10), ("p50", 50), ("p90", 90))},
+            "needle_recall": {"found": found, "planted": len(inp.needles),
+                              "recall": found / max(1, len(inp.needles))},
             "roofline": {"bound": "tensor", "kernel": "hga_attend",
                          "achieved": att_tflops, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": att_tflops / peak_tf,
