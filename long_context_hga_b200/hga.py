@@ -502,7 +502,11 @@ class KVStore:
     """History K/V in one file, read through a bounded page cache in host
     memory (pinned when a kernel gathers from it).  A page is page_tokens
     tokens of one KV head, K then V; the page table [Hkv][n_pages] maps a
-    page to its cache slot (-1 absent).  Wraps the hga_store_* calls."""
+    page to its cache slot (-1 absent).  Wraps the hga_store_* calls.
+
+    The cache and page table are tensors of this object that kernels read
+    in place: keep the object alive (and do not call reset_cache or
+    prepare) until every gather from it has completed on its stream."""
 
     def __init__(self, p: Params, path: str, t_cap: int, page_tokens: int, cache_pages: int,
                  create: bool = True, direct: bool = False, pin: bool = True):
