@@ -327,3 +327,61 @@ def test_argument_checks(hga, tmp_path):
     assert L.hga_store_length(None) == -1
     assert L.hga_store_close(None) == hga.HGA_OK
     assert _prepare(s, p, 64, 0, 64, gidx, gcnt)["pages_needed"] == 0
+
+
+def test_replacement_policy_over_many_random_steps(hga, tmp_path):
+    """Random steps over one history with a cache of about a third of it.
+    After every step: the step's pages are resident and hold their bytes,
+    residency never exceeds the cache, nothing leaves without a reason (a
+    resident page disappears only when the step had misses to place), and
+    eviction follows least-recent use by step: every evicted page was last
+    used no later than every retained page the step did not need."""
+    p, w = _params(hga, n_kv_heads=2, n_q_heads=4, top_chunks=4, top_groups=6, sink=64,
+                   local=64)
+    t_cap = 2048
+    q_starts = [1024, 1536, 1984]
+    k, v = _kv(w, 1024, 21)
+    pt = 8                                              # one group per page
+    hist_pages = w.n_kv_heads * 1024 // pt
+    s = _store(hga, p, tmp_path / "kv.bin", t_cap, cache_pages=hist_pages // 3,
+               page_tokens=pt)
+    s.append(k, v)
+    rng = np.random.default_rng(22)
+    last_use = {}
+    resident = set()
+    done = evictions = 0
+    for step in range(1, 41):
+        q_start = int(rng.choice(q_starts))
+        n_q = int(rng.integers(1, 3)) * 64 if q_start < 1984 else 64
+        n_q = min(n_q, t_cap - q_start)
+        gidx, gcnt = _routing(w, p, hga, q_start, n_q, 1024, 100 + step, t_cap)
+        need = _needed_pages(p, w, q_start, n_q, 1024, gidx, gcnt, pt)
+        if len(need) > s.cache_pages:
+            with pytest.raises(hga.HgaError) as e:
+                _prepare(s, p, q_start, n_q, 1024, gidx, gcnt)
+            assert e.value.code == hga.HGA_ERR_CAPACITY
+            continue
+        st = _prepare(s, p, q_start, n_q, 1024, gidx, gcnt, io_threads=3)
+        now = {(h, n) for h in range(w.n_kv_heads) for n in range(s.n_pages)
+               if s.page_table[h, n] >= 0}
+        assert need <= now and len(now) <= s.cache_pages
+        assert st["hits"] == len(need & resident)
+        assert st["misses"] == len(need - resident)
+        evicted = resident - now
+        assert now - need <= resident                     # no stray page appears
+        assert st["evictions"] == len(evicted)
+        if evicted:
+            assert st["misses"] > 0
+            kept_old = now - need
+            if kept_old:
+                assert max(last_use[x] for x in evicted) <= min(last_use[x] for x in kept_old)
+        for x in need:
+            last_use[x] = step
+        resident = now
+        done += 1
+        evictions += st["evictions"]
+        if step % 8 == 0:
+            _check_cache(s, w, k, v, need)
+    assert done >= 30 and evictions > 0, (done, evictions)
+    slots = s.page_table[s.page_table >= 0]
+    assert len(set(slots.tolist())) == len(slots)         # one page per slot
