@@ -385,3 +385,27 @@ def test_replacement_policy_over_many_random_steps(hga, tmp_path):
     assert done >= 30 and evictions > 0, (done, evictions)
     slots = s.page_table[s.page_table >= 0]
     assert len(set(slots.tolist())) == len(slots)         # one page per slot
+
+
+def test_fp32_store_with_head_dim_64(hga, tmp_path):
+    """The layout and the cache for 4-byte elements and d = 64."""
+    w = gi.TINY_FP32.with_(T=2048, q0=1536)
+    p = hga.Params.from_workload(w)
+    g = torch.Generator().manual_seed(31)
+    k = torch.randn(w.n_kv_heads, 1536, w.head_dim, generator=g)
+    v = torch.randn(w.n_kv_heads, 1536, w.head_dim, generator=g)
+    s = _store(hga, p, tmp_path / "kv.bin", w.T, cache_pages=64)
+    assert s.page_bytes == 2 * PT * w.head_dim * 4
+    s.append(k[:, :700], v[:, :700])
+    s.append(k[:, 700:], v[:, 700:])
+    rk, rv = s.read(5, 1530)
+    assert torch.equal(rk, k[:, 5:1530]) and torch.equal(rv, v[:, 5:1530])
+    gidx, gcnt = _routing(w, p, hga, w.q0, w.Tq, w.q0, 32, w.T)
+    need = _needed_pages(p, w, w.q0, w.Tq, w.q0, gidx, gcnt, PT)
+    st = _prepare(s, p, w.q0, w.Tq, w.q0, gidx, gcnt)
+    assert st["misses"] == len(need) > 0
+    cache = s.cache.view(torch.float32).view(s.cache_pages, 2, PT, w.head_dim)
+    for h, n in need:
+        slot = int(s.page_table[h, n])
+        assert torch.equal(cache[slot, 0], k[h, n * PT:(n + 1) * PT])
+        assert torch.equal(cache[slot, 1], v[h, n * PT:(n + 1) * PT])
