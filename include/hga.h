@@ -498,14 +498,39 @@ hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t s
  * operands; attention: 128 divisible by the query heads per KV head and at
  * most 4608 attended groups per block; routing: at most 8 query heads per KV
  * head and 4096 candidates per block), 1 = the portable mma.sync kernels,
- * 2 = same as 0, 3 = as 0 but attention with fp16 V and d = 128 runs on CTA
- * pairs (tcgen05.mma.cta_group::2, M = 256 over two SMs) when a block's rows
- * fill whole pairs of 256, the query heads per KV head are at least 2 and the
- * context is a multiple of the group size; it is correct but slower than the
- * one-CTA kernel on the measured workloads, hence not the default.  All
- * variants compute the same function; tests use the switch to check one
- * against another.  Returns HGA_ERR_INVALID_ARG for any other value. */
+ * 2 = same as 0.  All variants compute the same function; tests use the
+ * switch to check one against another.  Returns HGA_ERR_INVALID_ARG for any
+ * other value. */
 hga_status hga_set_kernel_variant(int32_t variant);
+
+/* ---------------------------------------------------------------------------
+ * Bounded waits.  Every wait of the tensor-core kernels (an mbarrier that a
+ * TMA copy, an MMA commit or another warp completes) gives up after a limit,
+ * raises HGA_ERR_TIMEOUT in the device status word (read by hga_check) and
+ * lets the kernel drain what it issued and return, so a lost completion never
+ * hangs the device.  No counterpart on the pages: this is the library's
+ * failure detection. */
+
+/* Sets the wait limit of the current device in nanoseconds (default 2e9,
+ * i.e. 2 s).  1e6 <= ns <= 6e10, else HGA_ERR_INVALID_ARG.  Synchronous; the
+ * limit applies to kernels launched afterwards on this device. */
+hga_status hga_set_wait_limit_ns(uint64_t ns);
+
+/* Self test of the bounded wait: one thread waits on an mbarrier that
+ * nothing arrives on.  It gives up after the current limit, sets
+ * HGA_ERR_TIMEOUT (returned by the next hga_check) and writes how long it
+ * waited, in ns, to *elapsed_ns (8 bytes of device memory owned by the
+ * caller).  Asynchronous on `stream`. */
+hga_status hga_selftest_wait(unsigned long long* elapsed_ns, hga_stream_t stream);
+
+/* Test hook (process-wide, one shot): the next launch of the tensor-core
+ * attention kernel stops its K/V loads at ring load `load_index` (0-based,
+ * counted over the CTA's K and V tiles in order), as if that copy never
+ * completed.  The kernel's waits on it run into the limit, the kernel
+ * returns and hga_check reports HGA_ERR_TIMEOUT; its output is then
+ * incomplete.  -1 clears the hook; other negative values give
+ * HGA_ERR_INVALID_ARG. */
+hga_status hga_debug_stall_next_attend(int64_t load_index);
 
 #ifdef __cplusplus
 }

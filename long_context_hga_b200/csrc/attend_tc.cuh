@@ -13,7 +13,8 @@
 // operand layout, so arbitrary group lists need no repacking.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q once, then K/V tiles into a 2-stage ring
+//   warp 0      TMA producer: Q first (before the group list is known), then
+//               K/V tiles into a 4-slot ring (one K or V tile per slot)
 //   warp 1      TMEM owner and MMA issuer (one thread):
 //                 S_i = Q_i K^T   (bf16 x bf16 -> fp32, K-major A and B)
 //                 O_i += P_i V    (fp16 P from TMEM x fp16 V, MN-major B)
@@ -46,6 +47,8 @@ constexpr float kTcRescaleLog2 = 8.0f;
 struct TcArgs {
   AttendArgs a;
   int rows_per_cta;                       // 256
+  int64_t stall_load;                     // test hook: the producer stops before this
+                                          // load of the ring (-1: never)
 };
 
 template <int D>
@@ -72,30 +75,56 @@ struct TcBars {
   int abort;
 };
 
-#ifdef HGA_TIMELINE
-// Debug builds only: SM clock stamps of pipeline events of CTA (0,0,0), kept
-// in shared memory (one region per role, no global round trips while the
-// kernel runs) and copied out at exit.
-__device__ unsigned long long g_tl[8192];
-__device__ unsigned int g_tl_n;
-__device__ unsigned long long g_cta[3 * 4096];   // per CTA: start ns, end ns, SM id
-struct TlBuf {
-  unsigned long long ev[5][128];
-  unsigned int n[5];
-  long long t0;
-};
-__device__ __forceinline__ void tl_mark(TlBuf* bf, int kind, int idx) {
-  if (blockIdx.x | blockIdx.y | blockIdx.z) return;
-  const int r = kind == 1 ? 0 : (kind <= 3 ? 1 : (kind == 4 || kind == 7 ? 2 : (threadIdx.x < 256 ? 3 : 4)));
-  const unsigned int k = atomicAdd(&bf->n[r], 1u);
-  if (k < 128)
-    bf->ev[r][k] = ((unsigned long long)(clock64() - bf->t0) << 16) | ((unsigned)kind << 10) |
-                   (unsigned)(idx & 1023);
+
+// The unit's group list (sink, routed, local window, diagonal; see
+// build_group_list) built by the whole CTA with one round of global reads:
+// every thread reads the routed entries its list slots would hold (and the
+// ones before them, for the ascending check) in the same round as the routed
+// count, instead of after it.  Invalid routed entries become -1 and are
+// reported; a list longer than the shared buffer gives 0 entries (reported).
+__device__ __forceinline__ int build_group_list_tc(const AttendArgs& a, int b, int h, int64_t b0,
+                                                   int64_t T, int* list, int* n_nondiag,
+                                                   bool* any_invalid) {
+  const int g = a.group;
+  const int64_t sink_end = min((int64_t)a.sink, b0);
+  const int n_s = (int)(sink_end / g);
+  const int32_t* routed = a.group_idx + ((int64_t)h * a.n_blocks + b) * a.cap_g;
+  const int64_t loc_lo = max(sink_end, b0 - a.local);
+  const int n_l = (int)((b0 - loc_lo) / g);
+  const int64_t b_end = min(b0 + a.qblock, T);
+  const int n_d = (int)((b_end - b0 + g - 1) / g);
+  const int n_max = (int)min((int64_t)a.max_list, (int64_t)n_s + a.cap_g + n_l + n_d);
+  int n_r = a.group_cnt[(int64_t)h * a.n_blocks + b];
+  const int64_t lo_tok = a.sink, hi_tok = b0 - a.local;
+  bool bad = false;
+  for (int i = threadIdx.x; i < n_max; i += blockDim.x) {
+    const int r = i - n_s;
+    const int cur = (r >= 0 && r < a.cap_g) ? routed[r] : -1;
+    const int prev = (r >= 1 && r <= a.cap_g) ? routed[r - 1] : -1;
+    int nr = n_r;
+    if (nr < 0 || nr > a.cap_g) nr = 0;
+    int e;
+    if (i < n_s) e = i;
+    else if (i < n_s + nr) {
+      e = cur;
+      const bool ok = (int64_t)e * g >= lo_tok && ((int64_t)e + 1) * g <= hi_tok &&
+                      (r == 0 || e > prev);
+      if (!ok) { e = -1; bad = true; }
+    } else if (i < n_s + nr + n_l) e = (int)(loc_lo / g) + (i - n_s - nr);
+    else if (i < n_s + nr + n_l + n_d) e = (int)(b0 / g) + (i - n_s - nr - n_l);
+    else continue;
+    list[i] = e;
+  }
+  if (n_r < 0 || n_r > a.cap_g) { bad = true; n_r = 0; }
+  if (bad) { report(HGA_ERR_DEVICE_CHECK); *any_invalid = true; }
+  const int n = n_s + n_r + n_l + n_d;
+  *n_nondiag = n_s + n_r + n_l;
+  if (n > a.max_list) {
+    if (threadIdx.x == 0) report(HGA_ERR_DEVICE_CHECK);
+    return 0;
+  }
+  return n;
 }
-#define HGA_TL(kind, idx) tl_mark(&s_tl, kind, idx)
-#else
-#define HGA_TL(kind, idx) ((void)0)
-#endif
 
 // The MMA issuer (one thread).  Per tile j it issues, for each Q tile i,
 // O_i += P_i(j-1) V(j-1) (once softmax has written P_i(j-1)) and then
@@ -104,22 +133,11 @@ __device__ __forceinline__ void tl_mark(TlBuf* bf, int kind, int idx) {
 // 64-bit add per MMA, and the tensor pipe stays fed only if nothing in this
 // loop waits on memory (inlined into the kernel, whose softmax code sets the
 // register allocation, the loop reloaded spilled values per MMA).
-#ifdef HGA_TIMELINE
-struct TlBuf;
-#define HGA_TLI(kind, idx) tl_mark(tlp, kind, idx)
-#else
-#define HGA_TLI(kind, idx) ((void)0)
-#endif
 template <int D>
 __device__ __noinline__ void tc_mma_issuer(TcBars* bars, uint32_t tmem, uint32_t q_base,
                                           uint32_t slot_base, int nq, int n_tiles,
-                                          volatile int* abort_flag, void* tl) {
+                                          volatile int* abort_flag) {
   using L = TcLayout<D>;
-#ifdef HGA_TIMELINE
-  TlBuf* tlp = static_cast<TlBuf*>(tl);
-#else
-  (void)tl;
-#endif
   constexpr uint32_t kIdS = tc::idesc_f16(kTcRows, kTcTok, 1, 0);
   constexpr uint32_t kIdPV = tc::idesc_f16(kTcRows, D, 0, 1);
   bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
@@ -145,7 +163,6 @@ __device__ __noinline__ void tc_mma_issuer(TcBars* bars, uint32_t tmem, uint32_t
           tc::mma_ts(d_o, a_p + k * 8, vd + (uint64_t)((2 * k * L::kGroupBytes) >> 4), kIdPV,
                      k > 0 ? 1u : acc0);
         tc::mma_commit(&bars->o_full[i]);
-        HGA_TLI(3, (j - 1) * 2 + i);
       }
       if (has_s) {
         if (i == 0) {
@@ -159,7 +176,6 @@ __device__ __noinline__ void tc_mma_issuer(TcBars* bars, uint32_t tmem, uint32_t
           tc::mma_ss(d_s, qd + (uint64_t)((((k >> 2) * L::kHalfBytes) + (k & 3) * 32) >> 4),
                      kd + (uint64_t)((((k >> 2) * 1024) + (k & 3) * 32) >> 4), kIdS, k > 0);
         tc::mma_commit(&bars->s_full[i]);
-        HGA_TLI(2, j * 2 + i);
       }
     }
     if (!ok) break;
@@ -172,7 +188,6 @@ __device__ __noinline__ void tc_mma_issuer(TcBars* bars, uint32_t tmem, uint32_t
   while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
   }
 }
-#undef HGA_TLI
 
 template <int D, bool VF16 = false>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -202,29 +217,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (row0 >= nrows) return;
   const int nq = (nrows - row0) > kTcRows ? 2 : 1;     // Q tiles with live rows
 
-  // ---- prologue: group list, barriers, TMEM
-  int n_nondiag;
-  bool inv = false;
-  if (tid == 0) bars->abort = 0;
-  const int n_list = build_group_list(a, b, h, b0, T, list, &n_nondiag, &inv);
-  if (n_list < 0) return;                       // uniform; reported inside
-  __shared__ int s_inv;
-  if (tid == 0) s_inv = 0;
-#ifdef HGA_TIMELINE
-  __shared__ TlBuf s_tl;
-  if (tid < 5) s_tl.n[tid] = 0;
-  if (tid == 0) s_tl.t0 = clock64();
-  const int cta_lin = (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
-  if (tid == 0 && cta_lin < 4096) {
-    unsigned int smid;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-    g_cta[3 * cta_lin] = tc::globaltimer_ns();
-    g_cta[3 * cta_lin + 2] = smid;
-  }
-#endif
-  __syncthreads();
-  if (inv) s_inv = 1;
+  // ---- prologue: barriers, the Q load, group list, TMEM.  Q depends on
+  // the unit only, so it is requested before the group list is read.
   if (tid == 0) {
+    bars->abort = 0;
     tc::mbar_init(&bars->q_full, 1);
     for (int s = 0; s < kTcSlots; ++s) {
       tc::mbar_init(&bars->full[s], 1);
@@ -241,6 +237,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc::mbar_init(&bars->ostage[1], kTcRows);
     tc::fence_mbar_init();
   }
+  __shared__ int s_inv;
+  if (tid == 0) s_inv = 0;
+  __syncthreads();
+  char* sQ = smem + L::kQOff;
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::tma_prefetch_desc(&tm_q);
+      tc::mbar_arrive_expect_tx(&bars->q_full, nq * L::kHalves * L::kHalfBytes);
+    }
+    __syncwarp();
+    if (lane < nq * L::kHalves) {
+      const int i = lane / L::kHalves, hf = lane % L::kHalves;
+      const int pos0 = (int)(b0 - a.q_start) + row0 / a.G;
+      tc::tma_load_3d(sQ + (i * L::kHalves + hf) * L::kHalfBytes, &tm_q, hf * 64, h * a.G,
+                      pos0 + i * (kTcRows / a.G), &bars->q_full);
+    }
+  }
+  int n_nondiag;
+  bool inv = false;
+  const int n_list = build_group_list_tc(a, b, h, b0, T, list, &n_nondiag, &inv);
+  if (inv) s_inv = 1;
   if (warp == 1) {
     tc::tmem_alloc(&bars->tmem_base, 512);
     tc::tmem_relinquish();
@@ -253,7 +270,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int n_tiles = (n_list + kTcGroupsPerTile - 1) / kTcGroupsPerTile;
   const int n_loads = 2 * n_tiles;             // K0 V0 K1 V1 ... through the ring
 
-  char* sQ = smem + L::kQOff;
   auto slot_ptr = [&](int s, int half) {
     return smem + L::kSlotOff + s * L::kSlotBytes + half * 1024;
   };
@@ -261,13 +277,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-#ifdef HGA_TIMELINE
-      void* tl = &s_tl;
-#else
-      void* tl = nullptr;
-#endif
       tc_mma_issuer<D>(bars, tmem, tc::smem_addr(sQ), tc::smem_addr(slot_ptr(0, 0)), nq, n_tiles,
-                       abort_flag, tl);
+                       abort_flag);
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -277,20 +288,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // tensor view (64 dims, 8 rows, 2 halves, group) lands as; 8 aligned
     // consecutive groups (sink, local window, diagonal, adjacent routed
     // groups) come in one 16 KB box.  Lane e < 16 owns entry e of the tile.
+    // (Q was requested in the prologue)
     if (lane == 0) {
-      tc::tma_prefetch_desc(&tm_q);
       tc::tma_prefetch_desc(&tm_k1);
       tc::tma_prefetch_desc(&tm_k8);
       tc::tma_prefetch_desc(&tm_v1);
       tc::tma_prefetch_desc(&tm_v8);
-      tc::mbar_arrive_expect_tx(&bars->q_full, nq * L::kHalves * L::kHalfBytes);
-    }
-    __syncwarp();
-    if (lane < nq * L::kHalves) {
-      const int i = lane / L::kHalves, hf = lane % L::kHalves;
-      const int pos0 = (int)(b0 - a.q_start) + row0 / a.G;
-      tc::tma_load_3d(sQ + (i * L::kHalves + hf) * L::kHalfBytes, &tm_q, hf * 64, h * a.G,
-                      pos0 + i * (kTcRows / a.G), &bars->q_full);
     }
     int last_use[kTcSlots];
 #pragma unroll
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int64_t head_group0 = (int64_t)h * (a.t_cap / a.group);
     for (int n = 0; n < n_loads; ++n) {
       const int s = n % kTcSlots, u = n / kTcSlots, j = n >> 1;
+      if (n == args.stall_load) break;      // test hook: this load is never issued
       int ok = 1;
       if (n >= kTcSlots && lane == 0) ok = tc::mbar_wait(&bars->empty[s], (u - 1) & 1, abort_flag);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
@@ -326,7 +330,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       last_use[s] = u;
-      if (lane == 0) HGA_TL(1, n);
     }
     // make sure no copy is still landing in shared memory when we leave
     if (lane == 0) {
@@ -354,8 +357,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     for (int j = 0; j < n_tiles; ++j) {
       const int nv = 2 * j + 1, s = nv % kTcSlots;
-      if (!tc::mbar_wait(&bars->full[s], (nv / kTcSlots) & 1, abort_flag)) break;
-      if (ct == 0) HGA_TL(4, j);
+      if (!tc::mbar_wait_warp(&bars->full[s], (nv / kTcSlots) & 1, abort_flag)) break;
       const int li0 = j * kTcGroupsPerTile;
       bool clean = li0 + kTcGroupsPerTile <= n_list && !any_invalid;
       if (clean) clean = ((int64_t)list[li0 + kTcGroupsPerTile - 1] + 1) * a.group <= T;
@@ -397,7 +399,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc::fence_proxy_async_smem();
       tc::mbar_arrive(&bars->v_ready[s]);
-      if (ct == 0) HGA_TL(7, j);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -413,8 +414,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float m = -INFINITY, l = 0.f;
     bool ok = i < nq;
     for (int j = 0; ok && j < n_tiles; ++j) {
-      if (!(ok = tc::mbar_wait(&bars->s_full[i], j & 1, abort_flag))) break;
-      if (tid == 128 || tid == 256) HGA_TL(5, j * 2 + i);
+      if (!(ok = tc::mbar_wait_warp(&bars->s_full[i], j & 1, abort_flag))) break;
       tc::fence_after_sync();
       // The whole S row (128 columns) is read from TMEM once, masked,
       // reduced to its max, then turned into P in place.
@@ -506,7 +506,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // O holds PV of tiles < j (PV of tile j waits for p_full below):
         // wait for the last one, then scale O in TMEM.  Done after P so the
         // S row's registers are free.
-        if (!(ok = tc::mbar_wait(&bars->o_full[i], (j - 1) & 1, abort_flag))) break;
+        if (!(ok = tc::mbar_wait_warp(&bars->o_full[i], (j - 1) & 1, abort_flag))) break;
         tc::fence_after_sync();
         const float f = rescale ? corr : 1.f;
 #pragma unroll
@@ -522,12 +522,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(&bars->p_full[i]);
-      if (tid == 128 || tid == 256) HGA_TL(6, j * 2 + i);
     }
     // ---- epilogue: O / l -> bf16, LSE
-    if (ok && i < nq && n_tiles > 0 && tc::mbar_wait(&bars->o_full[i], (n_tiles - 1) & 1, abort_flag)) {
+    if (ok && i < nq && n_tiles > 0 &&
+        tc::mbar_wait_warp(&bars->o_full[i], (n_tiles - 1) & 1, abort_flag)) {
       tc::fence_after_sync();
-      if (tid == 128 || tid == 256) HGA_TL(8, i);
       const float inv_l = 1.f / l;
       bool nonfinite = false;   // inf/NaN output: V outside the fp16 range (or bad input)
       // O / l as bf16 into this Q tile's shared memory (free once its last
@@ -572,7 +571,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         a.lse[(pos - a.q_start) * a.Hq + (int64_t)h * a.G + unit_row % a.G] =
             (m + log2f(l)) * 0.6931471805599453f;
       if (row_live && nonfinite) report(HGA_ERR_DEVICE_CHECK);
-      if (tid == 128 || tid == 256) HGA_TL(9, i);
     }
   }
 
@@ -584,15 +582,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, 512);
   }
-#ifdef HGA_TIMELINE
-  if (tid == 0 && cta_lin < 4096) g_cta[3 * cta_lin + 1] = tc::globaltimer_ns();
-  if (tid == 0 && !(blockIdx.x | blockIdx.y | blockIdx.z)) {
-    unsigned int k = 0;
-    for (int r = 0; r < 5; ++r)
-      for (unsigned int x = 0; x < min(s_tl.n[r], 128u) && k < 8192; ++x) g_tl[k++] = s_tl.ev[r][x];
-    g_tl_n = k;
-  }
-#endif
 }
 
 }  // namespace hga

@@ -15,6 +15,10 @@ __device__ int g_status;
 
 __device__ __forceinline__ void report(int code) { atomicCAS(&g_status, 0, code); }
 
+// Limit of every bounded wait of the tensor-core kernels, in nanoseconds
+// (2 s unless hga_set_wait_limit_ns changed it for the device).
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+
 // Programmatic dependent launch: every kernel of the library is launched so
 // that it may start while the previous kernel of the stream is finishing;
 // griddep_wait() blocks until that kernel has completed and its writes are

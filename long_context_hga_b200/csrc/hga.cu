@@ -16,7 +16,6 @@
 #include "route.cuh"
 #include "attend.cuh"
 #include "attend_tc.cuh"
-#include "attend_pair.cuh"
 #include "attend_bwd.cuh"
 #include "route_tc.cuh"
 #include "tier.cuh"
@@ -308,6 +307,10 @@ hga_status launch_summaries(const void* k, int64_t t_cap, int Hkv, int64_t t_beg
                     reinterpret_cast<__half*>(v_f16));
 }
 
+// One-shot test hook: the next tensor-core attention launch stops loading
+// K/V at this ring index (-1: off).  See hga_debug_stall_next_attend.
+std::atomic<int64_t> g_stall_next_attend{-1};
+
 template <int D, bool VF16>
 hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
   using L = hga::TcLayout<D>;
@@ -335,7 +338,10 @@ hga_status launch_attend_tc(hga::AttendArgs& a, cudaStream_t st) {
   if (!encode_bf16_map(&tk1, a.k, 4, gd, gs, b1) || !encode_bf16_map(&tk8, a.k, 4, gd, gs, b8) ||
       !encode_bf16_map(&tv1, a.v, 4, gd, gs, b1) || !encode_bf16_map(&tv8, a.v, 4, gd, gs, b8))
     return HGA_ERR_CUDA;
-  hga::TcArgs ta{a, 2 * hga::kTcRows};
+  hga::TcArgs ta{};
+  ta.a = a;
+  ta.rows_per_cta = 2 * hga::kTcRows;
+  ta.stall_load = g_stall_next_attend.exchange(-1, std::memory_order_relaxed);
   dim3 grid((a.qblock * a.G + ta.rows_per_cta - 1) / ta.rows_per_cta, a.n_blocks, a.Hkv);
   return launch_pdl(hga::attend_tc_kernel<D, VF16>, grid, dim3(hga::kTcThreads), smem, st, tq, tk1,
                     tk8, tv1, tv8, to, ta);
@@ -349,52 +355,9 @@ bool tc_eligible(const hga::AttendArgs& a) {
          a.n_q < (1ll << 31) && (a.t_cap % a.group) == 0;
 }
 
-// CTA-pair kernel (d = 128, fp16 V): 256 rows of a unit per pair, so the
-// unit's rows must fill whole pairs; every group in the lists must be whole
-// (context a multiple of the group size), since padding is zero-filled by
-// the loads rather than cleaned up; G >= 2 keeps one CTA's rows inside one
-// query block.
-bool pair_eligible(const hga::AttendArgs& a) {
-  return tc_eligible(a) && a.G >= 2 && ((int64_t)a.qblock * a.G) % 256 == 0 &&
-         ((a.q_start + a.n_q) % a.group) == 0 &&
-         (int64_t)a.Hkv * (a.t_cap / a.group) < (1ll << 31) - 1;
-}
-
-template <int D>
-hga_status launch_attend_pair(hga::AttendArgs& a, cudaStream_t st) {
-  const size_t smem = hga::pair_smem_bytes(a.max_list);
-  hga_status s = allow_smem<hga::attend_pair_kernel<D>>(smem);
-  if (s != HGA_OK) return s;
-  CUtensorMap tq, tk1, tk8, tv1, tv8, to;
-  const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
-  const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)a.Hq * D * 2};
-  const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(hga::kPrRows / a.G)};
-  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb) || !encode_bf16_map(&to, a.o, 3, qd, qs, qb))
-    return HGA_ERR_CUDA;
-  // K/V as (64 dims, 8 rows, D/64 halves, group).  K boxes carry both halves
-  // of a group; V boxes one half (the CTA's), so a V half tile lands as
-  // [group][8 rows][128 B].
-  const uint64_t gd[4] = {64, 8, (uint64_t)(D / 64), (uint64_t)a.Hkv * a.t_cap / 8};
-  const uint64_t gs[3] = {(uint64_t)D * 2, 128, (uint64_t)D * 2 * 8};
-  const uint32_t k1[4] = {64, 8, (uint32_t)(D / 64), 1};
-  const uint32_t k8[4] = {64, 8, (uint32_t)(D / 64), 8};
-  const uint32_t v1[4] = {64, 8, 1, 1};
-  const uint32_t v8[4] = {64, 8, 1, 8};
-  if (!encode_bf16_map(&tk1, a.k, 4, gd, gs, k1) || !encode_bf16_map(&tk8, a.k, 4, gd, gs, k8) ||
-      !encode_bf16_map(&tv1, a.v, 4, gd, gs, v1) || !encode_bf16_map(&tv8, a.v, 4, gd, gs, v8))
-    return HGA_ERR_CUDA;
-  const int pairs = (int)(((int64_t)a.qblock * a.G) / (2 * hga::kPrRows));
-  dim3 grid((unsigned)(2 * pairs), a.n_blocks, a.Hkv);
-  return launch_pdl(hga::attend_pair_kernel<D>, grid, dim3(hga::kPrThreads), smem, st, tq, tk1,
-                    tk8, tv1, tv8, to, a);
-}
-
 template <int D, bool VF16>
 hga_status launch_attend_bf16(hga::AttendArgs& a, cudaStream_t st) {
   const int variant = g_kernel_variant.load(std::memory_order_relaxed);
-  if constexpr (D == 128 && VF16) {
-    if (variant == 3 && pair_eligible(a)) return launch_attend_pair<D>(a, st);
-  }
   if (variant != 1 && tc_eligible(a)) return launch_attend_tc<D, VF16>(a, st);
   const size_t smem = hga::attend_mma_smem_bytes<D>(a.max_list);
   hga_status s = allow_smem<hga::attend_mma_kernel<D, VF16>>(smem);
@@ -725,44 +688,6 @@ const char* hga_status_string(hga_status s) {
 
 int64_t hga_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-#ifdef HGA_TIMELINE
-// Debug builds only (not part of the ABI): copies the attention kernel's
-// event stamps of CTA (0,0,0) and resets them; returns the count.
-int hga_debug_timeline(unsigned long long* out, int max) {
-  unsigned int n = 0, zero = 0;
-  cudaDeviceSynchronize();
-  cudaMemcpyFromSymbol(&n, hga::g_tl_n, sizeof(n));
-  if (n > 8192) n = 8192;
-  if ((int)n > max) n = (unsigned)max;
-  cudaMemcpyFromSymbol(out, hga::g_tl, n * sizeof(unsigned long long));
-  cudaMemcpyToSymbol(hga::g_tl_n, &zero, sizeof(zero));
-  return (int)n;
-}
-int hga_debug_route_times(unsigned long long* out, int max) {
-  cudaDeviceSynchronize();
-  const int n = max < 4 * 4096 ? max : 4 * 4096;
-  cudaMemcpyFromSymbol(out, hga::g_rt, n * sizeof(unsigned long long));
-  return n;
-}
-int hga_debug_pair_timeline(unsigned long long* out, int max) {
-  cudaDeviceSynchronize();
-  const int n = max < 2 * hga::kPrTlKinds * 128 ? max : 2 * hga::kPrTlKinds * 128;
-  cudaMemcpyFromSymbol(out, hga::g_pr_ev, n * sizeof(unsigned long long));
-  return n;
-}
-int hga_debug_pair_phases(unsigned long long* out, int max) {
-  cudaDeviceSynchronize();
-  const int n = max < 32 ? max : 32;
-  cudaMemcpyFromSymbol(out, hga::g_pr_ph, n * sizeof(unsigned long long));
-  return n;
-}
-int hga_debug_cta_times(unsigned long long* out, int max) {
-  cudaDeviceSynchronize();
-  const int n = max < 3 * 4096 ? max : 3 * 4096;
-  cudaMemcpyFromSymbol(out, hga::g_cta, n * sizeof(unsigned long long));
-  return n;
-}
-#endif
 
 // ---------------------------------------------------------------- host tier
 
@@ -946,12 +871,30 @@ hga_status hga_selftest_exp2(const float* x, float* y, int64_t n, hga_stream_t s
 }
 
 hga_status hga_set_kernel_variant(int32_t variant) {
-  if (variant < 0 || variant > 3) return HGA_ERR_INVALID_ARG;
+  if (variant < 0 || variant > 2) return HGA_ERR_INVALID_ARG;
   g_kernel_variant.store(variant, std::memory_order_relaxed);
   return HGA_OK;
 }
 
 const char* hga_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
+
+hga_status hga_set_wait_limit_ns(uint64_t ns) {
+  if (ns < 1000000ull || ns > 60000000000ull) return HGA_ERR_INVALID_ARG;
+  const unsigned long long v = ns;
+  return cuda_ok(cudaMemcpyToSymbol(hga::g_wait_limit_ns, &v, sizeof(v)));
+}
+
+hga_status hga_selftest_wait(unsigned long long* elapsed_ns, hga_stream_t stream) {
+  if (!elapsed_ns || (reinterpret_cast<uintptr_t>(elapsed_ns) & 7)) return HGA_ERR_INVALID_ARG;
+  hga::wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(elapsed_ns);
+  return after_launch();
+}
+
+hga_status hga_debug_stall_next_attend(int64_t load_index) {
+  if (load_index < -1) return HGA_ERR_INVALID_ARG;
+  g_stall_next_attend.store(load_index, std::memory_order_relaxed);
+  return HGA_OK;
+}
 
 }  // extern "C"
 

@@ -49,18 +49,6 @@ struct RtBars {
   int abort;
 };
 
-#ifdef HGA_TIMELINE
-// Debug builds only: per-CTA globaltimer stamps (start, scoring start,
-// scoring end, selection end).
-__device__ unsigned long long g_rt[4 * 4096];
-#define HGA_RT_STAMP(slot)                                                          \
-  do {                                                                              \
-    const int cta_l_ = blockIdx.y * gridDim.x + blockIdx.x;                         \
-    if (threadIdx.x == 0 && cta_l_ < 4096) g_rt[4 * cta_l_ + (slot)] = tc::globaltimer_ns(); \
-  } while (0)
-#else
-#define HGA_RT_STAMP(slot) ((void)0)
-#endif
 
 struct RtArgs {
   RouteArgs r;
@@ -250,7 +238,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  HGA_RT_STAMP(0);
   griddep_wait();
   const int b = blockIdx.x, h = blockIdx.y;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
@@ -284,7 +271,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   }
 
   // ---- scoring on the tensor cores
-  HGA_RT_STAMP(1);
   if (tid == 0) bars->abort = 0;
   if (warp == 1) {
     tc::tmem_alloc(&bars->tmem_base, 512);
@@ -299,9 +285,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   if (warp == 1) tc::tmem_dealloc(tmem, 512);
   if (*abort_flag) return;
   griddep_launch();
-  HGA_RT_STAMP(2);
   select_emit(sc, cd, k_eff, out, hist, tmp);
-  HGA_RT_STAMP(3);
 }
 
 struct RtFusedArgs {
@@ -333,7 +317,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  HGA_RT_STAMP(0);
   griddep_wait();
   const int b = blockIdx.x, h = blockIdx.y;
   const int64_t b0 = ac.q_start + (int64_t)b * ac.qblock;
@@ -379,7 +362,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   tc::fence_after_sync();
   const uint32_t tmem = bars[0].tmem_base;
   // ---- chunk scores and selection
-  HGA_RT_STAMP(1);
   if (score_c)
     rt_score<D>(&tm_q, &tm_c, true, ac, cc, args.rs, nrows, b0, h, smem, &bars[0], tmem, sc,
                 abort_flag);
@@ -403,9 +385,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   if ((score_c || score_g) && warp == 1) tc::tmem_dealloc(tmem, 512);
   if (*abort_flag) return;
   griddep_launch();
-  HGA_RT_STAMP(2);
   select_emit(sc, cg, k_g, out_g, hist, tmp);
-  HGA_RT_STAMP(3);
 }
 
 }  // namespace hga

@@ -45,26 +45,41 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Every wait in the tensor-core kernels is bounded: after kWaitLimitNs the
-// waiting thread raises the CTA's abort flag and the device status word
-// (HGA_ERR_TIMEOUT); any thread seeing the abort flag gives up too.  Returns
-// false when the wait did not complete.
+// Every wait in the tensor-core kernels is bounded: after the device's wait
+// limit (g_wait_limit_ns) the waiting thread raises the CTA's abort flag and
+// the device status word (HGA_ERR_TIMEOUT); any thread seeing the abort flag
+// gives up too.  Returns false when the wait did not complete.  The drains
+// that follow an abort (copies and MMAs already issued) wait at most
+// kWaitLimitNs each.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+
+__device__ __forceinline__ uint64_t wait_limit_ns() {
+  return *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns);
+}
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit) {
         *abort = 1;
         report(HGA_ERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+// mbar_wait by every lane of a warp, with one answer for the whole warp: a
+// lane whose wait ran out makes every lane give up, so warp-collective
+// instructions after the wait (tcgen05.ld/st) never see a split warp.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort));
 }
 
 // ---------------------------------------------------------------- TMA
@@ -107,6 +122,10 @@ __device__ __forceinline__ void bulk_commit_group() {
 // shared-memory source (the stores themselves complete asynchronously).
 __device__ __forceinline__ void bulk_wait_group_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory");
+}
+// Waits until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
 }
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* m, int x, int y, int z,
                                             int w, uint64_t* bar) {
@@ -244,6 +263,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort) {
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns();
   for (uint32_t i = 0;; ++i) {
     uint32_t ok;
     asm volatile(
@@ -255,7 +275,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if (ok) return true;
     if ((i & 31) == 31) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit) {
         *abort = 1;
         report(HGA_ERR_TIMEOUT);
         return false;
@@ -415,6 +435,23 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 }  // namespace tc
+
+// Bounded-wait self test: one thread waits on an mbarrier that nothing ever
+// arrives on.  The wait gives up after the device's wait limit, raising
+// HGA_ERR_TIMEOUT in the status word; *elapsed_ns receives how long it
+// waited.  No other thread, copy or MMA is involved, so the kernel always
+// ends.
+__global__ void wait_selftest_kernel(unsigned long long* elapsed_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  tc::mbar_init(&bar, 1);
+  tc::fence_mbar_init();
+  const uint64_t t0 = tc::globaltimer_ns();
+  const bool done = tc::mbar_wait(&bar, 0, &abort_flag);
+  *elapsed_ns = done ? 0ull : (unsigned long long)(tc::globaltimer_ns() - t0);
+}
 
 // y[i] = tc::exp2_fma2(x[i]) (pairs; a trailing odd element pairs with 0).
 __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y,

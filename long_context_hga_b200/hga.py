@@ -34,7 +34,8 @@ EXPORTED = ("hga_build_summaries", "hga_route_chunks", "hga_route_groups",
             "hga_attend_backward", "hga_decode_step", "hga_store_open", "hga_store_close",
             "hga_store_attach_cache", "hga_store_append", "hga_store_set_length",
             "hga_store_length", "hga_store_page_bytes", "hga_store_pages_per_head",
-            "hga_store_read", "hga_store_prepare", "hga_gather_store", "hga_forward_causal")
+            "hga_store_read", "hga_store_prepare", "hga_gather_store", "hga_forward_causal",
+            "hga_set_wait_limit_ns", "hga_selftest_wait", "hga_debug_stall_next_attend")
 
 
 class HgaError(RuntimeError):
@@ -106,6 +107,9 @@ def _load() -> ctypes.CDLL:
         "hga_last_cuda_error": [],
         "hga_set_kernel_variant": [i32],
         "hga_selftest_exp2": [vp, vp, i64, vp],
+        "hga_set_wait_limit_ns": [ctypes.c_uint64],
+        "hga_selftest_wait": [vp, vp],
+        "hga_debug_stall_next_attend": [i64],
         "hga_convert_v": [P, vp, i64, i64, i64, vp, vp],
         "hga_route": [P, vp, i64, i64, vp, vp, i64, vp, vp, vp, vp, vp],
         "hga_commit": [P, vp, vp, i64, i64, i64, vp, vp, vp, vp],
@@ -327,6 +331,27 @@ def selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
     _ok(LIB.hga_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
         "hga_selftest_exp2")
     return y
+
+
+def set_wait_limit_ns(ns: int):
+    """Limit of every bounded wait of the tensor-core kernels on the current
+    device (default 2e9 ns)."""
+    _ok(LIB.hga_set_wait_limit_ns(int(ns)), "hga_set_wait_limit_ns")
+
+
+def selftest_wait(stream=None) -> torch.Tensor:
+    """Runs the bounded-wait self test (a wait that nothing completes); returns
+    a device tensor holding how long it waited, in ns.  hga_check reports
+    HGA_ERR_TIMEOUT afterwards."""
+    out = torch.zeros(1, dtype=torch.int64, device="cuda")
+    _ok(LIB.hga_selftest_wait(_ptr(out), _stream(stream)), "hga_selftest_wait")
+    return out
+
+
+def debug_stall_next_attend(load_index: int):
+    """One-shot test hook: the next tensor-core attention launch stops its K/V
+    loads at this ring load, so its waits run into the limit (-1 clears)."""
+    _ok(LIB.hga_debug_stall_next_attend(int(load_index)), "hga_debug_stall_next_attend")
 
 
 # ---------------------------------------------------------------- host tier

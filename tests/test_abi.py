@@ -168,3 +168,14 @@ def test_product_path_has_no_oracle_import():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.replace("oracle)", ""), f
+
+
+def test_wait_hooks_reject_bad_arguments(hga):
+    """The bounded-wait controls refuse bad values before touching a device."""
+    assert hga.LIB.hga_set_wait_limit_ns(999_999) == hga.HGA_ERR_INVALID_ARG
+    assert hga.LIB.hga_set_wait_limit_ns(60_000_000_001) == hga.HGA_ERR_INVALID_ARG
+    assert hga.LIB.hga_selftest_wait(None, None) == hga.HGA_ERR_INVALID_ARG
+    assert hga.LIB.hga_selftest_wait(ctypes.c_void_p(12), None) == hga.HGA_ERR_INVALID_ARG
+    assert hga.LIB.hga_debug_stall_next_attend(-2) == hga.HGA_ERR_INVALID_ARG
+    assert hga.LIB.hga_debug_stall_next_attend(3) == hga.HGA_OK
+    assert hga.LIB.hga_debug_stall_next_attend(-1) == hga.HGA_OK      # cleared again

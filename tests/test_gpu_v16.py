@@ -121,9 +121,8 @@ CASES = {
 @pytest.mark.parametrize("variant", [2, 1])
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_fp16_v_gives_identical_attention(case, variant):
-    # variants 2 (same as the default, one CTA per SM) and 1: the fp16-V and
-    # bf16-V forms run the same arithmetic; the CTA-pair kernel (variant 3,
-    # fp16 V only) is checked against the oracle in test_gpu_parity.py
+    # variants 2 (same as the default tensor-core kernel) and 1 (mma.sync):
+    # the fp16-V and bf16-V forms run the same arithmetic
     hga = _hga()
     w = CASES[case]
     inp = gi.make_inputs(w)
