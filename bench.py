@@ -976,8 +976,10 @@ def measure_backward(w, dev, flush_w, flush_r, sink, reps=6):
     """Backward of the gathered attention (routing of the forward held fixed):
     device time of hga_attend_backward on the segment with a cold L2, and its
     algorithmic flops (10 d per (query row, attended token): the S and dP
-    products and the dQ, dK, dV accumulations) against the fp32 peak of the
-    CUDA cores, on which this first version runs."""
+    products and the dQ, dK, dV accumulations).  bf16 runs on the tensor
+    cores (against the bf16 peak); the fp32 CUDA-core kernel (variant 1) is
+    timed beside it on the same inputs.  The call also zeroes dK and dV on
+    the context's tokens (2 Hkv T d 4 bytes each), timed inside."""
     from long_context_hga_b200 import hga
     p = hga.Params.from_workload(w)
     inp = gi.make_inputs(w)
@@ -990,30 +992,49 @@ def measure_backward(w, dev, flush_w, flush_r, sink, reps=6):
     d_q = torch.empty(q.shape, dtype=torch.float32, device=dev)
     d_k = torch.empty(k.shape, dtype=torch.float32, device=dev)
     d_v = torch.empty(v.shape, dtype=torch.float32, device=dev)
-    ts = []
-    for i in range(reps + 2):
-        flush_w.zero_()
-        torch.sum(flush_r, 0, out=sink)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        hga.attend_backward(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse,
-                            d_o, d_q, d_k, d_v)
-        e1.record()
-        torch.cuda.synchronize()
-        if i >= 2:
-            ts.append(e0.elapsed_time(e1))
-    assert hga.check() == 0
+
+    def timed(variant):
+        hga.set_kernel_variant(variant)
+        try:
+            ts = []
+            for i in range(reps + 2):
+                flush_w.zero_()
+                torch.sum(flush_r, 0, out=sink)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                hga.attend_backward(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o,
+                                    bufs.lse, d_o, d_q, d_k, d_v)
+                e1.record()
+                torch.cuda.synchronize()
+                if i >= 2:
+                    ts.append(e0.elapsed_time(e1))
+        finally:
+            hga.set_kernel_variant(0)
+        assert hga.check() == 0
+        return float(np.median(ts))
+
     counts = algorithmic_counts(w, bufs.group_cnt.cpu().numpy())
     flops = counts["attn_flops"] * 10 / 4
-    ms = float(np.median(ts))
+    peaks, kind = load_peaks()
+    ms = timed(0)
+    ms_cc = timed(1) if w.dtype == "bf16" else None
     tf = flops / (ms * 1e-3) / 1e12
-    return {"workload": w.name, "backward": {
-        "ms": ms, "query_tokens_per_s": w.Tq / (ms * 1e-3),
-        "algorithmic_flops": flops, "tflops": tf,
-        "roofline": {"bound": "alu", "peak": FP32_ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
-                     "frac": tf / FP32_ALU_PEAK_TFLOPS,
-                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"},
-        "kernel": "fp32 CUDA cores, one CTA per 128-row slice, 16-byte atomics for dK/dV"}}
+    out = {"ms": ms, "query_tokens_per_s": w.Tq / (ms * 1e-3),
+           "algorithmic_flops": flops, "tflops": tf}
+    if w.dtype == "bf16":
+        out["roofline"] = {"bound": "tensor", "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                           "frac": tf / peaks["bf16_tflops"],
+                           "peak_source": f"{kind} bf16 burst"}
+        out["kernel"] = ("tcgen05: D = rowsum(dO o), dK/dV per (K/V tile, unit) with one "
+                         "float4 atomic flush per tile, dQ per 128-row tile")
+        out["fp32_cuda_core_kernel_ms"] = ms_cc
+    else:
+        out["roofline"] = {"bound": "alu", "peak": FP32_ALU_PEAK_TFLOPS, "unit": "TFLOP/s",
+                           "frac": tf / FP32_ALU_PEAK_TFLOPS,
+                           "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz"}
+        out["kernel"] = "fp32 CUDA cores, one CTA per 128-row slice, 16-byte atomics for dK/dV"
+    return {"workload": w.name, "backward": out}
 
 
 def measure_causal(w, dev, flush_w, flush_r, sink, reps=6):

@@ -17,6 +17,7 @@
 #include "attend.cuh"
 #include "attend_tc.cuh"
 #include "attend_bwd.cuh"
+#include "attend_bwd_tc.cuh"
 #include "route_tc.cuh"
 #include "tier.cuh"
 #include "noalloc.cuh"
@@ -388,6 +389,57 @@ hga_status launch_attend_bwd(hga::BwArgs& w, cudaStream_t st) {
   return launch_pdl(hga::attend_bwd_kernel<T, D>, grid, dim3(hga::kBwThreads), smem, st, w);
 }
 
+// Tensor-core backward (bf16): D = rowsum(dO o) into d_q's first column,
+// then the dK/dV kernel, then the dQ kernel (see attend_bwd_tc.cuh).  Every
+// group in the lists must be whole (the context a multiple of the group
+// size): a partial group's tokens past the context would be read from the
+// cache as they are.
+bool bwd_tc_eligible(const hga::AttendArgs& a, const void* o, const void* d_o) {
+  const uintptr_t align = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
+                          reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(o) |
+                          reinterpret_cast<uintptr_t>(d_o);
+  return (align & 15) == 0 && a.G <= hga::kBtRows && (hga::kBtRows % a.G) == 0 &&
+         a.max_list <= hga::kTcMaxList && (int64_t)a.Hkv * a.t_cap < (1ll << 31) &&
+         a.n_q < (1ll << 31) && (a.t_cap % a.group) == 0 && ((a.q_start + a.n_q) % a.group) == 0;
+}
+
+template <int D>
+hga_status launch_attend_bwd_tc(hga::BtArgs& w, cudaStream_t st) {
+  using LK = hga::BtKvLayout<D>;
+  using LQ = hga::BtQLayout<D>;
+  const hga::AttendArgs& a = w.a;
+  hga_status s = allow_smem<hga::bwd_dkdv_kernel<D>>(LK::smem_bytes());
+  if (s != HGA_OK) return s;
+  if ((s = allow_smem<hga::bwd_dq_kernel<D>>(LQ::smem_bytes(a.max_list))) != HGA_OK) return s;
+  CUtensorMap tq, tdo, tk1, tk8, tv1, tv8;
+  const uint64_t qd[3] = {(uint64_t)D, (uint64_t)a.Hq, (uint64_t)a.n_q};
+  const uint64_t qs[2] = {(uint64_t)D * 2, (uint64_t)a.Hq * D * 2};
+  const uint32_t qb[3] = {64, (uint32_t)a.G, (uint32_t)(hga::kBtRows / a.G)};
+  if (!encode_bf16_map(&tq, a.q, 3, qd, qs, qb) || !encode_bf16_map(&tdo, w.d_o, 3, qd, qs, qb))
+    return HGA_ERR_CUDA;
+  const uint64_t gd[4] = {64, 8, (uint64_t)(D / 64), (uint64_t)a.Hkv * a.t_cap / 8};
+  const uint64_t gs[3] = {(uint64_t)D * 2, 128, (uint64_t)D * 2 * 8};
+  const uint32_t b1[4] = {64, 8, (uint32_t)(D / 64), 1};
+  const uint32_t b8[4] = {64, 8, (uint32_t)(D / 64), 8};
+  if (!encode_bf16_map(&tk1, a.k, 4, gd, gs, b1) || !encode_bf16_map(&tk8, a.k, 4, gd, gs, b8) ||
+      !encode_bf16_map(&tv1, a.v, 4, gd, gs, b1) || !encode_bf16_map(&tv8, a.v, 4, gd, gs, b8))
+    return HGA_ERR_CUDA;
+  const int64_t n_rows = a.n_q * a.Hq;
+  const unsigned dblocks = (unsigned)std::min<int64_t>((n_rows + 7) / 8, 1 << 20);
+  if ((s = launch_pdl(hga::bwd_dsum_kernel<D>, dim3(dblocks), dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(w.o),
+                      static_cast<const __nv_bfloat16*>(w.d_o), w.d_q, n_rows)) != HGA_OK)
+    return s;
+  const int n_kv_tiles = (a.max_list + hga::kBtGroupsPerTile - 1) / hga::kBtGroupsPerTile;
+  dim3 gk((unsigned)n_kv_tiles, a.n_blocks, a.Hkv);
+  if ((s = launch_pdl(hga::bwd_dkdv_kernel<D>, gk, dim3(hga::kBtThreads), LK::smem_bytes(), st, tq,
+                      tdo, tk1, tk8, tv1, tv8, w)) != HGA_OK)
+    return s;
+  dim3 gq((unsigned)((a.qblock * a.G + hga::kBtRows - 1) / hga::kBtRows), a.n_blocks, a.Hkv);
+  return launch_pdl(hga::bwd_dq_kernel<D>, gq, dim3(hga::kBtThreads), LQ::smem_bytes(a.max_list),
+                    st, tq, tdo, tk1, tk8, tv1, tv8, w);
+}
+
 extern "C" {
 
 hga_status hga_validate_params(const hga_params* p) { return check_params(p); }
@@ -561,6 +613,21 @@ hga_status hga_attend_backward(const hga_params* p, const void* q, int64_t q_sta
   cudaError_t e = cudaMemset2DAsync(d_k, pitch, 0, row_bytes, p->n_kv_heads, st);
   if (e == cudaSuccess) e = cudaMemset2DAsync(d_v, pitch, 0, row_bytes, p->n_kv_heads, st);
   if (e != cudaSuccess) return cuda_ok(e);
+  if (p->dtype == HGA_BF16 && g_kernel_variant.load(std::memory_order_relaxed) != 1 &&
+      bwd_tc_eligible(a, o, d_o)) {
+    hga::BtArgs bt{};
+    bt.a = a;
+    bt.o = o;
+    bt.d_o = d_o;
+    bt.lse = lse;
+    bt.d_q = d_q;
+    bt.d_k = d_k;
+    bt.d_v = d_v;
+    bt.scale = w.scale;
+    bt.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->head_dim));
+    return p->head_dim == 128 ? launch_attend_bwd_tc<128>(bt, st)
+                              : launch_attend_bwd_tc<64>(bt, st);
+  }
   if (p->dtype == HGA_BF16)
     return p->head_dim == 128 ? launch_attend_bwd<__nv_bfloat16, 128>(w, st)
                               : launch_attend_bwd<__nv_bfloat16, 64>(w, st);
