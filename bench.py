@@ -889,6 +889,31 @@ def measure_all_configs(args, dev):
     return res
 
 
+def measure_one(name, args, dev):
+    """One per-workload measurement of measure_all_configs, alone."""
+    if name == "configs":
+        return measure_all_configs(args, dev)
+    flush_w = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_r = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    if name == "backward":
+        return measure_backward(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink)
+    if name == "tiered":
+        return measure_tiered(gi.TIERED_128K, dev, flush_w, flush_r, sink)
+    if name == "store":
+        return measure_store(gi.TIERED_128K, dev)
+    if name == "decode":
+        return measure_decode(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink)
+    if name == "causal":
+        return measure_causal(gi.QWEN3_30B_64K, dev, flush_w, flush_r, sink)
+    if name == "sweep":
+        inp = gi.make_inputs(gi.SWEEP_32K)
+        return [measure_config(gi.SWEEP_32K.with_(top_chunks=kc, top_groups=2 * kc), args, dev,
+                               flush_w, flush_r, sink, dense=False, inp=inp)[0]
+                for kc in gi.SWEEP_BUDGETS]
+    raise ValueError(name)
+
+
 def measure_decode(w, dev, flush_w, flush_r, sink, n_req=8, reps=6):
     """Generation steps at the 64K context: n_req requests, each with its own
     K/V cache (copies of the 64K workload's inputs), history committed; one
@@ -1155,6 +1180,10 @@ def main():
                     help="skip the brief per-workload report of the other configurations")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only", default=None,
+                    choices=["backward", "tiered", "store", "decode", "causal", "sweep", "configs"],
+                    help="run one of the per-workload measurements alone and print its "
+                         "JSON (for profiling); no headline line")
     ap.add_argument("--clock-window", type=float, default=0.6,
                     help="seconds of untimed replays on each side of the timed "
                          "region while nvidia-smi samples the clocks")
@@ -1162,6 +1191,9 @@ def main():
     if args.warmup < 3 and args.impl == "hga":
         args.warmup = 3
     world, rank, local = dist_setup()
+    if args.only is not None:
+        print(json.dumps(measure_one(args.only, args, torch.device("cuda", local))), flush=True)
+        return
     if args.impl == "reference":
         out = run_reference(args, world, rank)
     else:

@@ -242,8 +242,10 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start,
  * NULL), routes the block on the queries present and attends: one routing
  * decision per block, as in prefill (section 6.1 of the page), so the result
  * equals hga_forward of the segment [b0, pos + 1).  The token's output is row
- * pos - b0 of o ([n][Hq][d], n = pos - b0 + 1; earlier rows are recomputed
- * with the block's current routing).  chunk_idx .. group_cnt are sized for one
+ * pos - b0 of o ([n][Hq][d], n = pos - b0 + 1), and its LSE row pos - b0 of
+ * lse; the attention computes only the token's rows (bit for bit the rows
+ * hga_forward would give them), so the block's earlier rows of o and lse are
+ * left as they are.  chunk_idx .. group_cnt are sized for one
  * block; chunk_sum/group_sum hold the committed history.  params.v_f16 must be
  * 0 (v in dtype); v_f16 must not alias v.  Composed of the calls above; the
  * pages describe generation only in prose (section 2.2). */

@@ -32,6 +32,8 @@ struct AttendArgs {
   int n_blocks, Hq, Hkv, G;
   int group, qblock, sink, local;
   int max_list;           // group-list slots in shared memory
+  int64_t pos_lo;         // rows of positions before pos_lo may be skipped (their
+                          // outputs left as they are); q_start computes every row
   float scale_log2;       // log2(e) / sqrt(d)
 };
 

@@ -213,7 +213,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int64_t T = a.q_start + a.n_q;
   const int npos = (int)min((int64_t)a.qblock, T - b0);
   const int nrows = npos * a.G;
-  const int row0 = blockIdx.x * args.rows_per_cta;     // first unit row of this CTA
+  // first unit row of this CTA; rows of positions before pos_lo are skipped
+  const int skip = (int)min((int64_t)npos, max((int64_t)0, a.pos_lo - b0)) * a.G;
+  const int row0 = skip + blockIdx.x * args.rows_per_cta;
   if (row0 >= nrows) return;
   const int nq = (nrows - row0) > kTcRows ? 2 : 1;     // Q tiles with live rows
 

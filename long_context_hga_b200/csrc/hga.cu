@@ -440,6 +440,52 @@ hga_status launch_attend_bwd_tc(hga::BtArgs& w, cudaStream_t st) {
                     st, tq, tdo, tk1, tk8, tv1, tv8, w);
 }
 
+// hga_attend with rows of positions before pos_lo allowed to be skipped (the
+// tensor-core kernel skips them; the others compute every row).
+hga_status attend_impl(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
+                       const void* k, const void* v, int64_t t_cap, const int32_t* group_idx,
+                       const int32_t* group_cnt, void* o, float* lse, int64_t pos_lo,
+                       cudaStream_t st) {
+  hga_status s = check_params(p);
+  if (s != HGA_OK) return s;
+  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
+  if (n_q == 0) return HGA_OK;
+  if (!q || !k || !v || !group_idx || !group_cnt || !o) return HGA_ERR_INVALID_ARG;
+  hga::AttendArgs a{};
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.q_start = q_start;
+  a.n_q = n_q;
+  a.t_cap = t_cap;
+  a.group_idx = group_idx;
+  a.group_cnt = group_cnt;
+  a.cap_g = cap_groups(p, t_cap);
+  a.o = o;
+  a.lse = lse;
+  a.n_blocks = (int)((n_q + p->qblock - 1) / p->qblock);
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.G = p->n_q_heads / p->n_kv_heads;
+  a.group = p->group;
+  a.qblock = p->qblock;
+  a.sink = p->sink;
+  a.local = p->local;
+  const int64_t max_list = p->sink / p->group + a.cap_g + p->local / p->group +
+                           (p->qblock + p->group - 1) / p->group;
+  if (max_list > 16384) return HGA_ERR_UNSUPPORTED;
+  a.max_list = (int)max_list;
+  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->head_dim));
+  a.pos_lo = pos_lo;
+  if (p->dtype == HGA_BF16 && p->v_f16)
+    return p->head_dim == 128 ? launch_attend_bf16<128, true>(a, st)
+                              : launch_attend_bf16<64, true>(a, st);
+  if (p->dtype == HGA_BF16)
+    return p->head_dim == 128 ? launch_attend_bf16<128, false>(a, st)
+                              : launch_attend_bf16<64, false>(a, st);
+  return p->head_dim == 128 ? launch_attend_f32<128>(a, st) : launch_attend_f32<64>(a, st);
+}
+
 extern "C" {
 
 hga_status hga_validate_params(const hga_params* p) { return check_params(p); }
@@ -519,44 +565,8 @@ hga_status hga_route_groups(const hga_params* p, const void* q, int64_t q_start,
 hga_status hga_attend(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
                       const void* k, const void* v, int64_t t_cap, const int32_t* group_idx,
                       const int32_t* group_cnt, void* o, float* lse, hga_stream_t stream) {
-  hga_status s = check_params(p);
-  if (s != HGA_OK) return s;
-  if ((s = check_segment(p, q_start, n_q, t_cap)) != HGA_OK) return s;
-  if (n_q == 0) return HGA_OK;
-  if (!q || !k || !v || !group_idx || !group_cnt || !o) return HGA_ERR_INVALID_ARG;
-  hga::AttendArgs a{};
-  a.q = q;
-  a.k = k;
-  a.v = v;
-  a.q_start = q_start;
-  a.n_q = n_q;
-  a.t_cap = t_cap;
-  a.group_idx = group_idx;
-  a.group_cnt = group_cnt;
-  a.cap_g = cap_groups(p, t_cap);
-  a.o = o;
-  a.lse = lse;
-  a.n_blocks = (int)((n_q + p->qblock - 1) / p->qblock);
-  a.Hq = p->n_q_heads;
-  a.Hkv = p->n_kv_heads;
-  a.G = p->n_q_heads / p->n_kv_heads;
-  a.group = p->group;
-  a.qblock = p->qblock;
-  a.sink = p->sink;
-  a.local = p->local;
-  const int64_t max_list = p->sink / p->group + a.cap_g + p->local / p->group +
-                           (p->qblock + p->group - 1) / p->group;
-  if (max_list > 16384) return HGA_ERR_UNSUPPORTED;
-  a.max_list = (int)max_list;
-  a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p->head_dim));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (p->dtype == HGA_BF16 && p->v_f16)
-    return p->head_dim == 128 ? launch_attend_bf16<128, true>(a, st)
-                              : launch_attend_bf16<64, true>(a, st);
-  if (p->dtype == HGA_BF16)
-    return p->head_dim == 128 ? launch_attend_bf16<128, false>(a, st)
-                              : launch_attend_bf16<64, false>(a, st);
-  return p->head_dim == 128 ? launch_attend_f32<128>(a, st) : launch_attend_f32<64>(a, st);
+  return attend_impl(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, q_start,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 hga_status hga_attend_backward(const hga_params* p, const void* q, int64_t q_start, int64_t n_q,
@@ -725,8 +735,9 @@ hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos
     return s;
   hga_params pa = *p;
   pa.v_f16 = v_f16 ? 1 : 0;
-  return hga_attend(&pa, q_block, b0, n, k, v_f16 ? v_f16 : v, t_cap, group_idx, group_cnt, o,
-                    lse, stream);
+  // only the token's rows: the other rows of the block are not needed again
+  return attend_impl(&pa, q_block, b0, n, k, v_f16 ? v_f16 : v, t_cap, group_idx, group_cnt, o,
+                     lse, pos, reinterpret_cast<cudaStream_t>(stream));
 }
 
 hga_status hga_check(hga_stream_t stream) {

@@ -51,6 +51,7 @@ def test_decode_steps_match_oracle_and_prefill(v16):
                    pre.o, pre.lse)
         assert hga.check() == 0
         assert torch.equal(row, pre.o[n - 1])
+        assert torch.equal(bufs.lse[n - 1], pre.lse[n - 1])
         # the oracle on the context [0, pos + 1), segment [b0, pos + 1)
         qd, kd, vd = f(q_all[:n]), f(k[:, :pos + 1]), f(v[:, :pos + 1])
         res = ho.hga_forward(qd, kd, vd, b0, op)
