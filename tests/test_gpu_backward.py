@@ -136,3 +136,46 @@ def test_tensor_core_and_cuda_core_backward_agree():
     _check("tc", w, got_tc, ref, mag, 2.0 ** -8)
     _check("cuda_core", w, got_cc, ref, mag, 2.0 ** -16)
     assert not np.array_equal(got_tc[0], got_cc[0])     # two different kernels ran
+
+
+def test_backward_full_size_64k_sampled_dq():
+    """The 64K workload as the bench times it (tensor cores, fp16-free bf16
+    inputs): dq of sampled (block, KV head) units against the oracle's
+    backward of those units (a unit's dq depends on that unit alone)."""
+    from long_context_hga_b200 import hga
+    w = gi.QWEN3_30B_64K
+    p = hga.Params.from_workload(w)
+    inp = gi.make_inputs(w)
+    dev = torch.device("cuda:0")
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    bufs = hga.allocate(p, w.T, w.Tq, device=dev)
+    hga.build_summaries(p, k, 0, w.q0, bufs.chunk_sum, bufs.group_sum)
+    hga.forward(p, q, w.q0, k, v, bufs)
+    g = torch.Generator().manual_seed(17)
+    d_o = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+    d_q = torch.full(q.shape, float("nan"), dtype=torch.float32, device=dev)
+    d_k = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    d_v = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    hga.attend_backward(p, q, w.q0, k, v, bufs.group_idx, bufs.group_cnt, bufs.o, bufs.lse,
+                        d_o, d_q, d_k, d_v)
+    assert hga.check() == 0
+    f = lambda t: t.detach().to(torch.float64).cpu().numpy()
+    gi_np, gc_np = bufs.group_idx.cpu().numpy(), bufs.group_cnt.cpu().numpy()
+    op = ho.Params(w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.group, w.qblock,
+                   w.sink, w.local, w.top_chunks, w.top_groups, w.dtype)
+    qd, kd, vd, O, L, dO = f(q), f(k), f(v), f(bufs.o), f(bufs.lse), f(d_o)
+    got = f(d_q)
+    nb = w.Tq // w.qblock
+    units = [(0, 0), (nb - 1, w.n_kv_heads - 1), (nb // 2, 1), (7, 2), (nb - 5, 3)]
+    groups = {(b, h): [int(x) for x in gi_np[h, b, :gc_np[h, b]]] for (b, h) in units}
+    (Mq, _, _), (Eq, _, _) = _magnitudes(qd, kd, vd, w.q0, op, groups, O, L, dO)
+    for (b, h) in units:
+        r0, r1 = b * w.qblock, (b + 1) * w.qblock
+        hs = slice(h * w.G, (h + 1) * w.G)
+        dq, _, _ = ho.attend_unit_backward(qd, kd, vd, w.q0, w.T, groups[(b, h)], op, b, h,
+                                           O[r0:r1, hs], L[r0:r1, hs], dO[r0:r1, hs])
+        err = np.abs(got[r0:r1, hs] - dq)
+        bound = 2.0 ** -8 * Mq[r0:r1, hs] + w.head_dim * 2.0 ** -24 * Eq[r0:r1, hs] + 1e-7
+        worst = float(np.max(err / bound))
+        print("64k unit", (b, h), "max|err|", float(err.max()), "worst err/bound", worst)
+        assert worst <= 1.0, ((b, h), worst)
