@@ -190,10 +190,10 @@ __device__ __noinline__ void bt_kv_mma(BtKvBars* bars, uint32_t tmem, uint32_t k
   constexpr uint32_t kIdAcc = tc::idesc_f16(kBtTok, D, 1, 1);       // M tokens, N = d (MN-major B)
   const uint64_t k_desc = tc::sdesc_sw128(k_base, 16, L::kGroupBytes);
   const uint64_t v_desc = tc::sdesc_sw128(v_base, 16, L::kGroupBytes);
-  bool ok = tc::mbar_wait(&bars->kv_full, 0, abort_flag);
+  bool ok = tc::mbar_wait_warp(&bars->kv_full, 0, abort_flag);
   for (int rt = 0; ok && rt < n_rt; ++rt) {
     const int s = rt & 1;
-    if (!(ok = tc::mbar_wait(&bars->stage_full[s], (rt >> 1) & 1, abort_flag))) break;
+    if (!(ok = tc::mbar_wait_warp(&bars->stage_full[s], (rt >> 1) & 1, abort_flag))) break;
     tc::fence_after_sync();
     const uint32_t q_base = stage_base + s * 2 * L::kRowTileBytes;
     const uint32_t do_base = q_base + L::kRowTileBytes;
@@ -203,16 +203,16 @@ __device__ __noinline__ void bt_kv_mma(BtKvBars* bars, uint32_t tmem, uint32_t k
     for (int k = 0; k < D / 16; ++k) {
       const uint32_t ko = (uint32_t)(((k >> 2) * 1024 + (k & 3) * 32) >> 4);
       const uint32_t qo = (uint32_t)(((k >> 2) * L::kHalfBytes + (k & 3) * 32) >> 4);
-      tc::mma_ss(tmem + 0, k_desc + ko, q_kmaj + qo, kIdS, k > 0);        // S^T
+      tc::mma_ss_warp(tmem + 0, k_desc + ko, q_kmaj + qo, kIdS, k > 0);        // S^T
     }
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
       const uint32_t ko = (uint32_t)(((k >> 2) * 1024 + (k & 3) * 32) >> 4);
       const uint32_t qo = (uint32_t)(((k >> 2) * L::kHalfBytes + (k & 3) * 32) >> 4);
-      tc::mma_ss(tmem + 128, v_desc + ko, do_kmaj + qo, kIdS, k > 0);     // dP^T
+      tc::mma_ss_warp(tmem + 128, v_desc + ko, do_kmaj + qo, kIdS, k > 0);     // dP^T
     }
-    tc::mma_commit(&bars->sdp_full);
-    if (!(ok = tc::mbar_wait(&bars->p_full, rt & 1, abort_flag))) break;
+    tc::mma_commit_warp(&bars->sdp_full);
+    if (!(ok = tc::mbar_wait_warp(&bars->p_full, rt & 1, abort_flag))) break;
     tc::fence_after_sync();
     // B = dO or Q as [rows (K)][d (N)], N contiguous: halves L::kHalfBytes
     // apart, 8-row chunks 1 KB apart; one K step of 16 rows is 2 KB
@@ -220,16 +220,16 @@ __device__ __noinline__ void bt_kv_mma(BtKvBars* bars, uint32_t tmem, uint32_t k
     const uint64_t q_mn = tc::sdesc_sw128(q_base, L::kHalfBytes, 1024);
 #pragma unroll
     for (int k = 0; k < kBtRows / 16; ++k)
-      tc::mma_ts(tmem + 256, tmem + 0 + k * 8, do_mn + (uint64_t)((k * 2048) >> 4), kIdAcc,
-                 (rt > 0 || k > 0) ? 1u : 0u);                             // dV += P^T dO
+      tc::mma_ts_warp(tmem + 256, tmem + 0 + k * 8, do_mn + (uint64_t)((k * 2048) >> 4), kIdAcc,
+                      (rt > 0 || k > 0) ? 1u : 0u);                        // dV += P^T dO
 #pragma unroll
     for (int k = 0; k < kBtRows / 16; ++k)
-      tc::mma_ts(tmem + 384, tmem + 128 + k * 8, q_mn + (uint64_t)((k * 2048) >> 4), kIdAcc,
-                 (rt > 0 || k > 0) ? 1u : 0u);                             // dK += dS^T Q
-    tc::mma_commit(&bars->stage_empty[s]);
+      tc::mma_ts_warp(tmem + 384, tmem + 128 + k * 8, q_mn + (uint64_t)((k * 2048) >> 4), kIdAcc,
+                      (rt > 0 || k > 0) ? 1u : 0u);                        // dK += dS^T Q
+    tc::mma_commit_warp(&bars->stage_empty[s]);
   }
-  tc::mma_commit(&bars->acc_full);
-  tc::mma_commit(&bars->done);
+  tc::mma_commit_warp(&bars->acc_full);
+  tc::mma_commit_warp(&bars->done);
   const uint64_t t0 = tc::globaltimer_ns();
   while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
   }
@@ -291,9 +291,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   char* sStage = smem + L::kStage;
 
   if (warp == 1) {
-    if (lane == 0)
-      bt_kv_mma<D>(bars, tmem, tc::smem_addr(sK), tc::smem_addr(sV), tc::smem_addr(sStage), n_rt,
-                   abort_flag);
+    // the whole warp runs the issuer loop; elect.sync picks the issuing lane
+    bt_kv_mma<D>(bars, tmem, tc::smem_addr(sK), tc::smem_addr(sV), tc::smem_addr(sStage), n_rt,
+                 abort_flag);
   } else if (warp == 0) {
     // ---------------------------------------------------------- producer
     const int ent = bt_entry(lst, jt * kBtGroupsPerTile + (lane & 15), a.group);
@@ -472,10 +472,10 @@ __device__ __noinline__ void bt_q_mma(BtQBars* bars, uint32_t tmem, uint32_t q_b
   const uint64_t do_desc = tc::sdesc_sw128(do_base, 16, 1024);
   const uint64_t kv_kmaj0 = tc::sdesc_sw128(slot_base, 16, L::kGroupBytes);
   const uint64_t k_mn0 = tc::sdesc_sw128(slot_base, 1024, L::kGroupBytes);
-  bool ok = tc::mbar_wait(&bars->q_full, 0, abort_flag);
+  bool ok = tc::mbar_wait_warp(&bars->q_full, 0, abort_flag);
   for (int j = 0; ok && j < n_tiles; ++j) {
     const int nk = 2 * j, sk = nk % kTcSlots, nv = nk + 1, sv = nv % kTcSlots;
-    if (!(ok = tc::mbar_wait(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
+    if (!(ok = tc::mbar_wait_warp(&bars->full[sk], (nk / kTcSlots) & 1, abort_flag))) break;
     tc::fence_after_sync();
     const uint64_t kd = kv_kmaj0 + (uint64_t)((sk * L::kSlotBytes) >> 4);
     const uint64_t vd = kv_kmaj0 + (uint64_t)((sv * L::kSlotBytes) >> 4);
@@ -483,29 +483,30 @@ __device__ __noinline__ void bt_q_mma(BtQBars* bars, uint32_t tmem, uint32_t q_b
     for (int k = 0; k < D / 16; ++k) {
       const uint32_t ko = (uint32_t)(((k >> 2) * 1024 + (k & 3) * 32) >> 4);
       const uint32_t qo = (uint32_t)(((k >> 2) * L::kHalfBytes + (k & 3) * 32) >> 4);
-      tc::mma_ss(tmem + 0, q_desc + qo, kd + ko, kIdS, k > 0);            // S = Q K^T
+      tc::mma_ss_warp(tmem + 0, q_desc + qo, kd + ko, kIdS, k > 0);            // S = Q K^T
     }
-    if (!(ok = tc::mbar_wait(&bars->full[sv], (nv / kTcSlots) & 1, abort_flag))) break;
+    if (!(ok = tc::mbar_wait_warp(&bars->full[sv], (nv / kTcSlots) & 1, abort_flag))) break;
     tc::fence_after_sync();
 #pragma unroll
     for (int k = 0; k < D / 16; ++k) {
       const uint32_t ko = (uint32_t)(((k >> 2) * 1024 + (k & 3) * 32) >> 4);
       const uint32_t qo = (uint32_t)(((k >> 2) * L::kHalfBytes + (k & 3) * 32) >> 4);
-      tc::mma_ss(tmem + 128, do_desc + qo, vd + ko, kIdS, k > 0);         // dP = dO V^T
+      tc::mma_ss_warp(tmem + 128, do_desc + qo, vd + ko, kIdS, k > 0);         // dP = dO V^T
     }
-    tc::mma_commit(&bars->sdp_full);
-    if (!(ok = tc::mbar_wait(&bars->p_full, j & 1, abort_flag))) break;
+    tc::mma_commit_warp(&bars->sdp_full);
+    if (!(ok = tc::mbar_wait_warp(&bars->p_full, j & 1, abort_flag))) break;
     tc::fence_after_sync();
     const uint64_t kmn = k_mn0 + (uint64_t)((sk * L::kSlotBytes) >> 4);
 #pragma unroll
     for (int k = 0; k < kBtTok / 16; ++k)
-      tc::mma_ts(tmem + 256, tmem + 0 + k * 8, kmn + (uint64_t)((2 * k * L::kGroupBytes) >> 4),
-                 kIdQ, (j > 0 || k > 0) ? 1u : 0u);                        // dQ += dS K
-    tc::mma_commit(&bars->empty[sk]);
-    tc::mma_commit(&bars->empty[sv]);
+      tc::mma_ts_warp(tmem + 256, tmem + 0 + k * 8,
+                      kmn + (uint64_t)((2 * k * L::kGroupBytes) >> 4), kIdQ,
+                      (j > 0 || k > 0) ? 1u : 0u);                         // dQ += dS K
+    tc::mma_commit_warp(&bars->empty[sk]);
+    tc::mma_commit_warp(&bars->empty[sv]);
   }
-  tc::mma_commit(&bars->dq_full);
-  tc::mma_commit(&bars->done);
+  tc::mma_commit_warp(&bars->dq_full);
+  tc::mma_commit_warp(&bars->done);
   const uint64_t t0 = tc::globaltimer_ns();
   while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
   }
@@ -586,9 +587,9 @@ __global__ void __launch_bounds__(kBtThreads, 1)
   auto slot_ptr = [&](int s) { return smem + L::kSlot + s * L::kSlotBytes; };
 
   if (warp == 1) {
-    if (lane == 0)
-      bt_q_mma<D>(bars, tmem, tc::smem_addr(sQ), tc::smem_addr(sDO), tc::smem_addr(slot_ptr(0)),
-                  n_tiles, abort_flag);
+    // the whole warp runs the issuer loop; elect.sync picks the issuing lane
+    bt_q_mma<D>(bars, tmem, tc::smem_addr(sQ), tc::smem_addr(sDO), tc::smem_addr(slot_ptr(0)),
+                n_tiles, abort_flag);
   } else if (warp == 0) {
     // ---------------------------------------------------------- producer
     // ring load n: K of tile n/2 (n even) or V (n odd), into slot n % 4

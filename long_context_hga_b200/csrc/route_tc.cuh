@@ -142,18 +142,20 @@ __device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool 
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ------------------------------------------------------------ MMA
+      // the whole warp runs the loop; elect.sync picks the issuing lane
       const uint32_t idesc = tc::idesc_f16(kRtTile, RS, 1, 0);
       const uint32_t q_base = tc::smem_addr(sQ);
-      bool ok = !load_q || tc::mbar_wait(&bars->q_full, 0, abort_flag);
+      bool ok = !load_q || tc::mbar_wait_warp(&bars->q_full, 0, abort_flag);
       for (int t = 0; ok && t < n_tiles; ++t) {
         const int s = t & 1;
-        if (!(ok = tc::mbar_wait(&bars->full[s], (t >> 1) & 1, abort_flag))) break;
+        if (!(ok = tc::mbar_wait_warp(&bars->full[s], (t >> 1) & 1, abort_flag))) break;
         tc::fence_after_sync();
         for (int r = 0; r < n_slices; ++r) {
           const int q = t * n_slices + r, buf = q & 1;
-          if (q >= 2 && !(ok = tc::mbar_wait(&bars->acc_empty[buf], ((q >> 1) - 1) & 1, abort_flag)))
+          if (q >= 2 &&
+              !(ok = tc::mbar_wait_warp(&bars->acc_empty[buf], ((q >> 1) - 1) & 1, abort_flag)))
             break;
           tc::fence_after_sync();
           // base descriptors once; k-steps move only the start address
@@ -161,14 +163,15 @@ __device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool 
           const uint64_t bd0 = tc::sdesc_sw128(q_base + r * L::kHalves * L::kQHalf, 16, 1024);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
-            tc::mma_ss(tmem + buf * 256,
-                       ad0 + (uint64_t)((((k >> 2) * L::kTileHalf) + (k & 3) * 32) >> 4),
-                       bd0 + (uint64_t)((((k >> 2) * L::kQHalf) + (k & 3) * 32) >> 4), idesc, k > 0);
-          tc::mma_commit(&bars->acc_full[buf]);
+            tc::mma_ss_warp(tmem + buf * 256,
+                            ad0 + (uint64_t)((((k >> 2) * L::kTileHalf) + (k & 3) * 32) >> 4),
+                            bd0 + (uint64_t)((((k >> 2) * L::kQHalf) + (k & 3) * 32) >> 4), idesc,
+                            k > 0);
+          tc::mma_commit_warp(&bars->acc_full[buf]);
         }
-        if (ok) tc::mma_commit(&bars->empty[s]);
+        if (ok) tc::mma_commit_warp(&bars->empty[s]);
       }
-      tc::mma_commit(&bars->done);
+      tc::mma_commit_warp(&bars->done);
       const uint64_t t0 = tc::globaltimer_ns();
       while (!tc::mbar_try_wait(&bars->done, 0) && tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
       }
