@@ -337,7 +337,12 @@ def run_hga(args, world, rank, local):
     # segment's own tokens are converted inside every step) or bf16 (each
     # attention tile is converted on chip)
     v16 = args.v_storage == "f16"
-    p_att = dataclasses.replace(p, v_f16=True) if v16 else p
+    # q_ready: the routing and attention calls below each follow one of the
+    # library's own kernels in the stream (the step starts with commit), and
+    # those let the next kernel start only after their own wait, so q is
+    # complete by then and may be requested before that wait
+    pq = dataclasses.replace(p, q_ready=True)
+    p_att = dataclasses.replace(pq, v_f16=True) if v16 else pq
     v_att = torch.empty(v.shape, dtype=torch.float16, device=dev) if v16 else v
     # commit the history once (setup, not timed)
     hga.commit(p, k, v, 0, w.q0, bufs.chunk_sum, bufs.group_sum, v_att if v16 else None)
@@ -353,14 +358,14 @@ def run_hga(args, world, rank, local):
                             v_att if v16 else None)),
     ] + ([
         ("route",
-         lambda: hga.route(p, q, w.q0, bufs.chunk_sum, bufs.group_sum, w.T, bufs.chunk_idx,
+         lambda: hga.route(pq, q, w.q0, bufs.chunk_sum, bufs.group_sum, w.T, bufs.chunk_idx,
                            bufs.chunk_cnt, bufs.group_idx, bufs.group_cnt)),
     ] if args.route == "fused" else [
         ("route_chunks",
-         lambda: hga.route_chunks(p, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx,
+         lambda: hga.route_chunks(pq, q, w.q0, bufs.chunk_sum, w.T, bufs.chunk_idx,
                                   bufs.chunk_cnt)),
         ("route_groups",
-         lambda: hga.route_groups(p, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx,
+         lambda: hga.route_groups(pq, q, w.q0, bufs.group_sum, w.T, bufs.chunk_idx,
                                   bufs.chunk_cnt, bufs.group_idx, bufs.group_cnt)),
     ]) + [
         ("attend",
@@ -485,8 +490,8 @@ def run_hga(args, world, rank, local):
             if i >= 2:
                 s_cmp.wait_event(ev_out[x])         # step i-2's O has been read back
             hga.commit(p, kb, vb, w.q0, w.T, bb.chunk_sum, bb.group_sum, vab if v16 else None)
-            hga.route_chunks(p, q_d, w.q0, bb.chunk_sum, w.T, bb.chunk_idx, bb.chunk_cnt)
-            hga.route_groups(p, q_d, w.q0, bb.group_sum, w.T, bb.chunk_idx, bb.chunk_cnt,
+            hga.route_chunks(pq, q_d, w.q0, bb.chunk_sum, w.T, bb.chunk_idx, bb.chunk_cnt)
+            hga.route_groups(pq, q_d, w.q0, bb.group_sum, w.T, bb.chunk_idx, bb.chunk_cnt,
                              bb.group_idx, bb.group_cnt)
             hga.attend(p_att, q_d, w.q0, kb, vab, bb.group_idx, bb.group_cnt, bb.o, bb.lse)
             ev_cmp[x].record(s_cmp)

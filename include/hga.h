@@ -99,6 +99,20 @@ typedef struct hga_params {
                         /* P, 11 significant bits), so they read V as is     */
                         /* instead of converting each tile; dtype must be    */
                         /* HGA_BF16.  hga_convert_v fills such a buffer.     */
+  int32_t q_ready;      /* 0 or 1.  Every kernel of this library is launched */
+                        /* with programmatic dependent launch: it may start  */
+                        /* while the kernel before it in the stream is still */
+                        /* running, and waits for that kernel before reading */
+                        /* its inputs.  1 promises that q is complete before */
+                        /* that kernel can let its dependents start (kernels */
+                        /* that never do so early, such as PyTorch's, and    */
+                        /* this library's own kernels qualify); the          */
+                        /* tensor-core routing and attention kernels then    */
+                        /* request q before the wait, overlapping its load   */
+                        /* with the previous kernel's tail.  0: q is read    */
+                        /* after the wait.  hga_forward, hga_forward_causal  */
+                        /* and hga_decode_step use 1 for their own calls     */
+                        /* that follow one of their kernels.                 */
 } hga_params;
 
 /* Step 1 (section 2.1, "HGA builds two levels of key summaries from the

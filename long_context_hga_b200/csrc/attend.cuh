@@ -35,6 +35,7 @@ struct AttendArgs {
   int64_t pos_lo;         // rows of positions before pos_lo may be skipped (their
                           // outputs left as they are); q_start computes every row
   float scale_log2;       // log2(e) / sqrt(d)
+  int q_early;            // q may be requested before waiting for the previous kernel
 };
 
 // Builds the unit's group list in shared memory; returns the entry count and

@@ -211,7 +211,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* list = reinterpret_cast<int*>(smem + L::kListOff);
   volatile int* abort_flag = &bars->abort;
 
-  griddep_wait();
+  // Every input is read after waiting for the previous kernel, except Q with
+  // q_early (complete before that kernel can let this one start): its load
+  // is then requested first and overlaps that kernel's tail.
+  if (!a.q_early) griddep_wait();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.y, h = blockIdx.z;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
@@ -261,6 +264,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       pos0 + i * (kTcRows / a.G), &bars->q_full);
     }
   }
+  if (a.q_early) griddep_wait();
   int n_nondiag;
   bool inv = false;
   const int n_list = build_group_list_tc(a, b, h, b0, T, list, &n_nondiag, &inv);

@@ -99,6 +99,7 @@ hga_status check_params(const hga_params* p) {
   if (p->dtype != HGA_BF16 && p->dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
   if (p->v_f16 != 0 && p->v_f16 != 1) return HGA_ERR_INVALID_ARG;
   if (p->v_f16 && p->dtype != HGA_BF16) return HGA_ERR_INVALID_ARG;
+  if (p->q_ready != 0 && p->q_ready != 1) return HGA_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return HGA_ERR_UNSUPPORTED;
   if (p->chunk != 64 || p->group != 8 || p->qblock != 64) return HGA_ERR_UNSUPPORTED;
   return HGA_OK;
@@ -166,7 +167,8 @@ bool route_tc_eligible(const hga::RouteArgs& a, const void* q, const void* summ)
 template <int D>
 hga_status launch_route_tc(hga::RouteArgs& a, cudaStream_t st) {
   using L = hga::RtLayout<D>;
-  hga_status s = allow_smem<hga::route_tc_kernel<D>>(L::kSmem);
+  hga_status s = a.q_early ? allow_smem<hga::route_tc_kernel<D, true>>(L::kSmem)
+                           : allow_smem<hga::route_tc_kernel<D, false>>(L::kSmem);
   if (s != HGA_OK) return s;
   hga::RtArgs ra{a, std::min(256, 64 * a.G)};
   CUtensorMap tq, ts, ts8;
@@ -181,8 +183,11 @@ hga_status launch_route_tc(hga::RouteArgs& a, cudaStream_t st) {
       !encode_bf16_map(&ts8, a.summ, 2, sd, ss, sb8))
     return HGA_ERR_CUDA;
   dim3 grid(a.n_blocks, a.Hkv);
-  return launch_pdl(hga::route_tc_kernel<D>, grid, dim3(hga::kRtThreads), L::kSmem, st, tq, ts,
-                    ts8, ra);
+  if (a.q_early)
+    return launch_pdl(hga::route_tc_kernel<D, true>, grid, dim3(hga::kRtThreads), L::kSmem, st,
+                      tq, ts, ts8, ra);
+  return launch_pdl(hga::route_tc_kernel<D, false>, grid, dim3(hga::kRtThreads), L::kSmem, st, tq,
+                    ts, ts8, ra);
 }
 
 template <int D>
@@ -247,6 +252,7 @@ hga_status route_args(const hga_params* p, const void* q, int64_t q_start, int64
   a.sink = p->sink;
   a.local = p->local;
   a.group_mode = group_mode;
+  a.q_early = p->q_ready;
   a.in_idx = in_idx;
   a.in_cnt = in_cnt;
   a.out_idx = out_idx;
@@ -471,6 +477,7 @@ hga_status attend_impl(const hga_params* p, const void* q, int64_t q_start, int6
   a.qblock = p->qblock;
   a.sink = p->sink;
   a.local = p->local;
+  a.q_early = p->q_ready;
   const int64_t max_list = p->sink / p->group + a.cap_g + p->local / p->group +
                            (p->qblock + p->group - 1) / p->group;
   if (max_list > 16384) return HGA_ERR_UNSUPPORTED;
@@ -680,10 +687,12 @@ hga_status hga_forward(const hga_params* p, const void* q, int64_t q_start, int6
   if (s != HGA_OK) return s;
   s = hga_route_chunks(p, q, q_start, n_q, chunk_sum, t_cap, chunk_idx, chunk_cnt, stream);
   if (s != HGA_OK) return s;
-  s = hga_route_groups(p, q, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+  hga_params pq = *p;     // these follow the library's own routing kernels
+  pq.q_ready = 1;
+  s = hga_route_groups(&pq, q, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
                        group_cnt, stream);
   if (s != HGA_OK) return s;
-  return hga_attend(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
+  return hga_attend(&pq, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
 }
 
 hga_status hga_forward_causal(const hga_params* p, const void* q_ext, int64_t q_start,
@@ -707,10 +716,12 @@ hga_status hga_forward_causal(const hga_params* p, const void* q_ext, int64_t q_
   if ((s = hga_route_chunks(p, q_ext, q_start, n_q, chunk_sum, t_cap, chunk_idx, chunk_cnt,
                             stream)) != HGA_OK)
     return s;
-  if ((s = hga_route_groups(p, q_ext, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt,
+  hga_params pq = *p;     // these follow the library's own routing kernels
+  pq.q_ready = 1;
+  if ((s = hga_route_groups(&pq, q_ext, q_start, n_q, group_sum, t_cap, chunk_idx, chunk_cnt,
                             group_idx, group_cnt, stream)) != HGA_OK)
     return s;
-  return hga_attend(p, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
+  return hga_attend(&pq, q, q_start, n_q, k, v, t_cap, group_idx, group_cnt, o, lse, stream);
 }
 
 hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos, const void* k,
@@ -730,10 +741,12 @@ hga_status hga_decode_step(const hga_params* p, const void* q_block, int64_t pos
   if ((s = hga_route_chunks(p, q_block, b0, n, chunk_sum, t_cap, chunk_idx, chunk_cnt, stream)) !=
       HGA_OK)
     return s;
-  if ((s = hga_route_groups(p, q_block, b0, n, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
+  hga_params pq = *p;     // these follow the library's own routing kernels
+  pq.q_ready = 1;
+  if ((s = hga_route_groups(&pq, q_block, b0, n, group_sum, t_cap, chunk_idx, chunk_cnt, group_idx,
                             group_cnt, stream)) != HGA_OK)
     return s;
-  hga_params pa = *p;
+  hga_params pa = pq;
   pa.v_f16 = v_f16 ? 1 : 0;
   // only the token's rows: the other rows of the block are not needed again
   return attend_impl(&pa, q_block, b0, n, k, v_f16 ? v_f16 : v, t_cap, group_idx, group_cnt, o,

@@ -41,6 +41,7 @@ struct RouteArgs {
   int top_k;              // <= 0: all
   int group_mode;         // 0: chunk candidates, 1: groups of kept chunks
   int max_cands;          // shared-memory score slots
+  int q_early;            // q may be requested before waiting for the previous kernel
 };
 
 // ---------------------------------------------------------------- block scan
@@ -520,6 +521,11 @@ __device__ void select_emit(const float* sc, const Cands& cd, int k_eff, int32_t
 __device__ int compact_kept_chunks(const RouteArgs& a, int b, int h, int lo, int64_t hi,
                                    int* kept, int* s_n, int* tmp) {
   const int32_t* in = a.in_idx + ((int64_t)h * a.n_blocks + b) * a.in_cap;
+  // the first round's entries are read in the same round as the count (the
+  // row holds in_cap slots, so these reads stay inside it whatever the count)
+  const int lim = (int)min(a.in_cap, (int64_t)2048);
+  const int c_first = threadIdx.x < lim ? in[threadIdx.x] : -1;
+  const int p_first = threadIdx.x >= 1 && threadIdx.x - 1 < lim ? in[threadIdx.x - 1] : -1;
   int cnt = a.in_cnt[(int64_t)h * a.n_blocks + b];
   if (cnt < 0 || cnt > a.in_cap || cnt > 2048) {
     if (threadIdx.x == 0) report(HGA_ERR_DEVICE_CHECK);
@@ -531,8 +537,8 @@ __device__ int compact_kept_chunks(const RouteArgs& a, int b, int h, int lo, int
     int c = -1;
     bool ok = false;
     if (i < cnt) {
-      c = in[i];
-      const int prev = i > 0 ? in[i - 1] : -1;
+      c = i0 == 0 ? c_first : in[i];
+      const int prev = i > 0 ? (i0 == 0 ? p_first : in[i - 1]) : -1;
       ok = c >= lo && c < hi && c > prev;
       if (!ok) report(HGA_ERR_DEVICE_CHECK);
     }

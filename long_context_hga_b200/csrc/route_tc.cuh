@@ -57,12 +57,13 @@ struct RtArgs {
 
 // Scores every candidate of `cd` for the unit (block at b0, KV head h):
 // sc[i] = max over the unit's rows of q_row . summary(cd.id(i)).  Warp 0
-// streams the summaries (and Q first when load_q; otherwise Q is already in
-// shared memory), warp 1 issues the MMAs into the double-buffered TMEM
+// streams the summaries (and Q first when load_q, unless q_issued: the caller
+// then initialised q_full and requested Q itself; without load_q Q is already
+// in shared memory), warp 1 issues the MMAs into the double-buffered TMEM
 // accumulator at `tmem`, warps 4-7 reduce each candidate's row maxima.  Uses
 // the barrier set `bars` (initialised here) and ends with a CTA barrier.
 template <int D>
-__device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool load_q,
+__device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool load_q, bool q_issued,
                          const RouteArgs& a, const Cands& cd, int RS, int nrows, int64_t b0,
                          int h, char* smem, RtBars* bars, uint32_t tmem, float* sc,
                          volatile int* abort_flag) {
@@ -72,7 +73,7 @@ __device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool 
   const int n_tiles = (cd.n + kRtTile - 1) / kRtTile;
   const int n_jobs = n_tiles * n_slices;
   if (tid == 0) {
-    tc::mbar_init(&bars->q_full, 1);
+    if (!q_issued) tc::mbar_init(&bars->q_full, 1);
     for (int s = 0; s < 2; ++s) {
       tc::mbar_init(&bars->full[s], 1);
       tc::mbar_init(&bars->empty[s], 1);
@@ -96,7 +97,7 @@ __device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool 
     // half (lane e < 16 issues kept chunk e of the tile).
     if (lane == 0) {
       tc::tma_prefetch_desc(tm_s);
-      if (load_q) {
+      if (load_q && !q_issued) {
         tc::tma_prefetch_desc(tm_q);
         const int pos0 = (int)(b0 - a.q_start);
         tc::mbar_arrive_expect_tx(&bars->q_full, n_slices * L::kHalves * RS * 128);
@@ -221,8 +222,10 @@ __device__ void rt_score(const CUtensorMap* tm_q, const CUtensorMap* tm_s, bool 
   tc::fence_after_sync();
 }
 
-// Chunk routing or group routing of one (query block, KV head) unit.
-template <int D>
+// Chunk routing or group routing of one (query block, KV head) unit.  QE:
+// the call's q_early (a compile-time choice, so that the default form is
+// built without the early-copy code).
+template <int D, bool QE>
 __global__ void __launch_bounds__(kRtThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_s,
@@ -241,11 +244,35 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __shared__ int tmp[32 + 256];          // scan slots + second histogram buffer
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  griddep_wait();
   const int b = blockIdx.x, h = blockIdx.y;
   const int64_t b0 = a.q_start + (int64_t)b * a.qblock;
   const int npos = (int)min((int64_t)a.qblock, a.q_start + a.n_q - b0);
   const int nrows = npos * a.G;
+  // With q_early, Q (an input of the call, complete before the previous
+  // kernel can let this one start) is requested before waiting for that
+  // kernel, so its load overlaps the previous kernel's tail; exits that score
+  // nothing then wait for that copy first.
+  constexpr bool q_issued = QE;
+  if (QE && tid == 0) {
+    const int RS = args.rs, n_slices = (nrows + RS - 1) / RS;
+    tc::mbar_init(&bars->q_full, 1);
+    tc::fence_mbar_init();
+    tc::tma_prefetch_desc(&tm_q);
+    tc::mbar_arrive_expect_tx(&bars->q_full, n_slices * L::kHalves * RS * 128);
+    for (int r = 0; r < n_slices; ++r)
+      for (int hf = 0; hf < L::kHalves; ++hf)
+        tc::tma_load_3d(smem + (r * L::kHalves + hf) * L::kQHalf, &tm_q, hf * 64, h * a.G,
+                        (int)(b0 - a.q_start) + r * (RS / a.G), &bars->q_full);
+  }
+  auto drain_q = [&]() {
+    if (QE && tid == 0) {
+      const uint64_t t0 = tc::globaltimer_ns();
+      while (!tc::mbar_try_wait(&bars->q_full, 0) &&
+             tc::globaltimer_ns() - t0 < tc::kWaitLimitNs) {
+      }
+    }
+  };
+  griddep_wait();
 
   // ---- candidates (same rules as route_kernel)
   Cands cd;
@@ -263,13 +290,18 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   int32_t* out = a.out_idx + ((int64_t)h * a.n_blocks + b) * a.out_cap;
   if (k_eff > a.out_cap || cd.n > kRtMaxCands) {
     if (tid == 0) report(HGA_ERR_DEVICE_CHECK);
+    drain_q();
     return;
   }
   for (int i = k_eff + tid; i < a.out_cap; i += kRtThreads) out[i] = -1;
   if (tid == 0) a.out_cnt[(int64_t)h * a.n_blocks + b] = k_eff;
-  if (k_eff == 0) return;
+  if (k_eff == 0) {
+    drain_q();
+    return;
+  }
   if (k_eff >= cd.n) {          // every candidate kept: no scores needed
     select_emit(sc, cd, k_eff, out, hist, tmp);
+    drain_q();
     return;
   }
 
@@ -283,7 +315,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
-  rt_score<D>(&tm_q, a.group_mode ? &tm_s8 : &tm_s, true, a, cd, args.rs, nrows, b0, h, smem, bars,
+  rt_score<D>(&tm_q, a.group_mode ? &tm_s8 : &tm_s, true, q_issued, a, cd, args.rs, nrows, b0, h, smem, bars,
               tmem, sc, abort_flag);
   if (warp == 1) tc::tmem_dealloc(tmem, 512);
   if (*abort_flag) return;
@@ -366,7 +398,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   const uint32_t tmem = bars[0].tmem_base;
   // ---- chunk scores and selection
   if (score_c)
-    rt_score<D>(&tm_q, &tm_c, true, ac, cc, args.rs, nrows, b0, h, smem, &bars[0], tmem, sc,
+    rt_score<D>(&tm_q, &tm_c, true, false, ac, cc, args.rs, nrows, b0, h, smem, &bars[0], tmem, sc,
                 abort_flag);
   if (*abort_flag) {
     if ((score_c || score_g) && warp == 1) tc::tmem_dealloc(tmem, 512);
@@ -383,7 +415,7 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   cg.lo = cc.lo;
   cg.n = n_g;
   if (score_g)
-    rt_score<D>(&tm_q, &tm_g8, !score_c, ag, cg, args.rs, nrows, b0, h, smem, &bars[1], tmem, sc,
+    rt_score<D>(&tm_q, &tm_g8, !score_c, false, ag, cg, args.rs, nrows, b0, h, smem, &bars[1], tmem, sc,
                 abort_flag);
   if ((score_c || score_g) && warp == 1) tc::tmem_dealloc(tmem, 512);
   if (*abort_flag) return;

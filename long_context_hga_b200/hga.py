@@ -47,7 +47,7 @@ class HgaError(RuntimeError):
 class CParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "n_q_heads", "n_kv_heads", "head_dim", "chunk", "group", "qblock",
-        "sink", "local", "top_chunks", "top_groups", "dtype", "v_f16")]
+        "sink", "local", "top_chunks", "top_groups", "dtype", "v_f16", "q_ready")]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -65,13 +65,14 @@ class Params:
     top_groups: int = 8
     dtype: str = "bf16"
     v_f16: bool = False          # v holds fp16 values (see convert_v)
+    q_ready: bool = False        # q complete before the previous kernel can let this one start
 
     def c(self) -> CParams:
         return CParams(self.n_q_heads, self.n_kv_heads, self.head_dim,
                        self.chunk, self.group, self.qblock, self.sink,
                        self.local, self.top_chunks, self.top_groups,
                        HGA_BF16 if self.dtype == "bf16" else HGA_FP32,
-                       int(self.v_f16))
+                       int(self.v_f16), int(self.q_ready))
 
     @property
     def torch_dtype(self):

@@ -60,6 +60,11 @@ def test_param_validation(hga):
     bad = ok.c()
     bad.v_f16 = 2
     assert hga.LIB.hga_validate_params(ctypes.byref(bad)) == hga.HGA_ERR_INVALID_ARG
+    # q_ready is a promise about the stream (0 or 1)
+    assert hga.validate_params(P(32, 4, 128, q_ready=True)) == 0
+    bad = ok.c()
+    bad.q_ready = -1
+    assert hga.LIB.hga_validate_params(ctypes.byref(bad)) == hga.HGA_ERR_INVALID_ARG
 
 
 def test_index_capacity(hga):

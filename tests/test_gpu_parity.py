@@ -202,3 +202,40 @@ def test_fused_route_equals_two_calls(case):
     assert hga.check() == 0
     assert torch.equal(a.chunk_cnt, b.chunk_cnt) and torch.equal(a.chunk_idx, b.chunk_idx)
     assert torch.equal(a.group_cnt, b.group_cnt) and torch.equal(a.group_idx, b.group_idx)
+
+
+@pytest.mark.parametrize("case", ["30b_ragged", "budget_all", "g16", "d64_g1"])
+def test_q_ready_calls_equal_the_default(case):
+    """With q_ready the routing and attention kernels request q before waiting
+    for the previous kernel (each call here follows one of the library's own
+    kernels, as the promise requires).  Their outputs equal the default
+    path's bit for bit; the full budget takes the routing exits that score
+    nothing (and must wait for that early copy before leaving)."""
+    import dataclasses
+    from long_context_hga_b200 import hga
+    w = {"30b_ragged": gi.QWEN3_30B_64K.with_(T=4136, q0=2048, n_needles=8),
+         "budget_all": gi.SWEEP_32K.with_(T=4096, q0=2048, top_chunks=0, top_groups=0),
+         "g16": gi.Workload("g16", 16, 1, 128, 1600, 1024, 1e6, 128, 128, 5, 12, n_needles=4),
+         "d64_g1": gi.Workload("d64_g1", 4, 4, 64, 1536, 512, 1e6, 64, 128, 3, 10,
+                               n_needles=4)}[case]
+    p = hga.Params.from_workload(w)
+    pr = dataclasses.replace(p, q_ready=True)
+    inp = gi.make_inputs(w)
+    dev = torch.device("cuda:0")
+    q, k, v = inp.q.to(dev), inp.k.to(dev), inp.v.to(dev)
+    out = []
+    for pp in (p, pr):
+        bb = hga.allocate(p, w.T, w.Tq, device=dev)
+        bb.o.fill_(float("nan"))
+        hga.commit(p, k, v, 0, w.T, bb.chunk_sum, bb.group_sum)
+        for _ in range(2):          # the second pass starts right after the first's attention
+            hga.route_chunks(pp, q, w.q0, bb.chunk_sum, w.T, bb.chunk_idx, bb.chunk_cnt)
+            hga.route_groups(pp, q, w.q0, bb.group_sum, w.T, bb.chunk_idx, bb.chunk_cnt,
+                             bb.group_idx, bb.group_cnt)
+            hga.attend(pp, q, w.q0, k, v, bb.group_idx, bb.group_cnt, bb.o, bb.lse)
+        assert hga.check() == 0
+        out.append(bb)
+    a, b = out
+    for name in ("chunk_cnt", "chunk_idx", "group_cnt", "group_idx", "o", "lse"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    assert torch.isfinite(b.o.float()).all()
